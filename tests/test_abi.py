@@ -1,0 +1,87 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/tpconv.h declares, plans match the oracle's path table,
+the device CG table (Racah construction) agrees with the oracle's independent
+null-space construction, errors are reported, workspace is edge-independent."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import workloads as W
+from oracle import conv, so3
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def T():
+    from equivariant_gnn_tensor_receiver_b200 import build
+    build.build(verbose=False)
+    import equivariant_gnn_tensor_receiver_b200 as T
+    return T
+
+
+def test_exports_every_declared_symbol(T):
+    hdr = open(os.path.join(ROOT, "include", "tpconv.h")).read()
+    declared = set(re.findall(r"\b(tpconv_\w+)\s*\(", hdr))
+    assert declared == set(T.exported_names())
+    L = ctypes.CDLL(T._lib.LIB_PATH)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+@pytest.mark.parametrize("name", ["tiny", "mace", "sweep", "wide"])
+def test_plan_matches_oracle_path_table(T, name):
+    c = W.CONFIGS[name]
+    plan = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], radial=c["radial"],
+                  radial_params=c["radial_params"])
+    prob = conv.Problem(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], c["radial"], c["radial_params"])
+    assert plan.n_paths == len(prob.paths)
+    assert (plan.dim_in, plan.dim_out, plan.n_sh, plan.theta_numel) == (prob.dim_in, prob.dim_out, prob.n_sh,
+                                                                          prob.theta_numel)
+    for a, p in zip(plan.paths, prob.paths):
+        assert (a["l1"], a["l2"], a["l3"], a["c_in"], a["c_out"], a["theta_offset"]) == (
+            p.l1, p.l2, p.l3, p.c_in, p.c_out, p.theta_off)
+
+
+def test_cg_table_matches_null_space_construction(T):
+    worst = 0.0
+    for l1 in range(4):
+        for l2 in range(4):
+            for l3 in range(abs(l1 - l2), min(l1 + l2, 3) + 1):
+                got = T.tpconv_cg_coefficients(l1, l2, l3)
+                want = so3.real_cg(l1, l2, l3)
+                worst = max(worst, np.abs(got - want).max())
+    assert worst < 1e-12
+
+
+def test_errors_are_reported(T):
+    with pytest.raises(T.TPConvError) as e:
+        T.Plan("8x0e+8xe", 1, "8x0e", 4)
+    assert e.value.status == 2
+    with pytest.raises(T.TPConvError) as e:
+        T.Plan("8x4e", 1, "8x0e", 4)
+    assert e.value.status == 3
+    with pytest.raises(T.TPConvError) as e:
+        T.Plan("8x0e", 4, "8x0e", 4)
+    assert e.value.status == 3
+    with pytest.raises(T.TPConvError) as e:
+        T.Plan("8x0e", 1, "8x0e", 17)
+    assert e.value.status == 3
+    with pytest.raises(T.TPConvError) as e:
+        T.tpconv_cg_coefficients(1, 1, 3)
+    assert e.value.status == 3
+
+
+def test_workspace_independent_of_edges_and_capped(T):
+    c = W.CONFIGS["mace"]
+    plan = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"])
+    sizes = {T.tpconv_workspace_size(plan, op, 4096, E) for op in (0,) for E in (10, 10 ** 6, 10 ** 8)}
+    assert len(sizes) == 1
+    cap = 64 << 20
+    capped = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], workspace_cap=cap)
+    for op in (0, 1, 2):
+        assert T.tpconv_workspace_size(capped, op, 1_222_309, 64_000_000) < cap + (16 << 20)
