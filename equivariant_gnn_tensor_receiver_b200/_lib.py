@@ -56,7 +56,13 @@ _EXPORTS = {
     "tpconv_forward": (ctypes.c_int, [_P, _I64, _I64] + [_P] * 6 + [_P, ctypes.c_size_t, _P]),
     "tpconv_backward": (ctypes.c_int, [_P, _I64, _I64] + [_P] * 14 + [_P, ctypes.c_size_t, _P]),
     "tpconv_double_backward": (ctypes.c_int, [_P, _I64, _I64] + [_P] * 16 + [_P, ctypes.c_size_t, _P]),
+    "tpconv_profile_enable": (ctypes.c_int, [ctypes.c_int]),
+    "tpconv_profile_reset": (ctypes.c_int, []),
+    "tpconv_profile_read": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_double),
+                                           ctypes.POINTER(ctypes.c_int64)]),
 }
+PHASES = ["transpose", "fwd_edge", "fwd_node", "bwd_node_g", "bwd_edge_r", "bwd_edge_s", "bwd_node_x",
+          "dbl_edge_a", "dbl_node_a", "dbl_edge_r", "dbl_edge_s", "dbl_node_x", "other"]
 
 
 def exported_names():
@@ -219,3 +225,23 @@ def tpconv_double_backward(plan, N, E, rowptr, col, perm, s_rowptr, s_recv, edge
                                         _ptr(gg_vec, f32), _ptr(gg_theta, f32), _ptr(d_g, f32),
                                         _ptr(d_x, f32), _ptr(d_vec, f32), _ptr(d_theta, f32), w, wb,
                                         _stream(stream)))
+
+
+def tpconv_profile_enable(on: bool = True):
+    _check("tpconv_profile_enable", lib().tpconv_profile_enable(int(bool(on))))
+
+
+def tpconv_profile_reset():
+    _check("tpconv_profile_reset", lib().tpconv_profile_reset())
+
+
+def tpconv_profile_read(phase: int):
+    """(device milliseconds, kernel launches) of one phase since the last reset."""
+    ms = ctypes.c_double()
+    n = ctypes.c_int64()
+    _check("tpconv_profile_read", lib().tpconv_profile_read(int(phase), ctypes.byref(ms), ctypes.byref(n)))
+    return ms.value, n.value
+
+
+def profile_all():
+    return {name: tpconv_profile_read(i) for i, name in enumerate(PHASES)}

@@ -334,14 +334,21 @@ int tpconv_plan_create(tpconv_plan** out, const char* irreps_in, int l_sh_max,
       }
   d.P = P;
   d.rm = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
-  int sm = 0;
+  int sm = 0, sm2 = 0;
   for (int i = 0; i < P; ++i) {
     DevPath& q = d.path[i];
     q.nmz = m_count(q.l1, q.l2, q.l3);
     q.sm_off = sm;
     sm += kEdgeBatch * (q.nmz + 2 * d.rm + 1 + (2 * q.l2 + 1));
+    q.sm_off2 = sm2;
+    sm2 += kEdgeBatch * (2 * q.nmz + 4 * d.rm + 1 + 2 * (2 * q.l2 + 1));
   }
   d.sm_floats = sm;
+  d.sm_floats2 = sm2;
+  if (size_t(std::max(sm, sm2)) * 4 > 227 * 1024) {
+    delete p;
+    return TPCONV_ERR_UNSUPPORTED;
+  }
   d.a_pref[0] = 0;
   for (int i3 = 0; i3 < d.n_out; ++i3) d.a_pref[i3 + 1] = d.a_pref[i3] + int64_t(2 * d.out_l[i3] + 1) * d.Kb[i3];
   d.b_pref[0] = 0;

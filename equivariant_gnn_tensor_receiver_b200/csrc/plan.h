@@ -92,7 +92,8 @@ struct DevPath {
   int32_t kxoff;            // B column of (k=0, w=0) in input block i1: kxoff + k*c_out + w
   int64_t theta_off;        // start of Theta[p] ([R][c_in][c_out])
   int32_t nmz;              // m_count(l1, l2, l3)
-  int32_t sm_off;           // float offset of this path's warp scratch in dynamic smem
+  int32_t sm_off;           // float offset of this path's warp scratch (first-order adjoint stream)
+  int32_t sm_off2;          // same for the double-backward adjoint stream
 };
 
 struct DevPlan {
@@ -108,7 +109,8 @@ struct DevPlan {
   int64_t b_pref[kMaxBlocks + 1];   // floats per node before block i1 (sum n1 * Kx)
   int max_c_in, max_c_out;
   int rm;                           // radial registers per lane (4, 8 or 16) >= R
-  int sm_floats;                    // dynamic smem floats of the edge-stream kernels
+  int sm_floats;                    // dynamic smem floats of the first-order adjoint stream
+  int sm_floats2;                   // dynamic smem floats of the double-backward adjoint stream
   DevPath path[kMaxPaths];
 };
 

@@ -13,8 +13,10 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "gemm_simt.cuh"
 #include "graph.cuh"
@@ -40,11 +42,48 @@ int ensure_device() {
   if (g_ready[dev]) return TPCONV_OK;
   const float* t = cg_table_f32();
   if (!t) return TPCONV_ERR_INTERNAL;
-  if (upload_cg_fwd(t) || upload_cg_send(t) || upload_cg_radj(t)) return TPCONV_ERR_CUDA;
-  if (radj_set_smem_limit(227 * 1024)) return TPCONV_ERR_CUDA;
+  if (upload_cg_fwd(t) || upload_cg_send(t) || upload_cg_radj(t) || upload_cg_dbl(t)) return TPCONV_ERR_CUDA;
+  if (radj_set_smem_limit(227 * 1024) || dbl_set_smem_limit(227 * 1024)) return TPCONV_ERR_CUDA;
   g_ready[dev] = true;
   return TPCONV_OK;
 }
+
+// ---- diagnostics: per-phase launch counts and optional event timing ----
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pending[TPCONV_N_PHASES];
+  double ms[TPCONV_N_PHASES] = {};
+  std::atomic<int64_t> launches[TPCONV_N_PHASES];
+  Profiler() {
+    for (auto& l : launches) l = 0;
+  }
+};
+Profiler& prof() {
+  static Profiler p;
+  return p;
+}
+inline void note(int phase, int64_t n) { prof().launches[phase] += n; }
+
+// Brackets one phase of a call with events on the call's stream (when enabled).
+struct PhaseScope {
+  int phase;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr, b = nullptr;
+  PhaseScope(int ph, cudaStream_t s) : phase(ph), st(s) {
+    Profiler& p = prof();
+    if (!p.on) return;
+    if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) return;
+    cudaEventRecord(a, st);
+  }
+  ~PhaseScope() {
+    if (!b) return;
+    cudaEventRecord(b, st);
+    Profiler& p = prof();
+    std::lock_guard<std::mutex> lk(p.mu);
+    p.pending[phase].push_back({a, b});
+  }
+};
 
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 inline float* F(const float* p) { return const_cast<float*>(p); }
@@ -63,9 +102,9 @@ int check_ws(const tpconv_plan* plan, int op, int64_t N, int64_t E, void* ws, si
   return TPCONV_OK;
 }
 
-// out[r0 : r0+nc] = A . Theta  (per output block)
+// out[r0 : r0+nc] = A . Theta (mode 0) or += (mode 1), per output block
 cudaError_t node_mix_forward(const DevPlan& d, int r0, int nc, const float* A, const float* theta, float* out,
-                             cudaStream_t st) {
+                             cudaStream_t st, int mode = 0) {
   for (int i3 = 0; i3 < d.n_out; ++i3) {
     const int n3 = 2 * d.out_l[i3] + 1, cout = d.out_mul[i3];
     const int p0 = first_path_of_out_block(d, i3);
@@ -73,7 +112,7 @@ cudaError_t node_mix_forward(const DevPlan& d, int r0, int nc, const float* A, c
     MView a = mrow(F(A) + size_t(nc) * d.a_pref[i3], d.Kb[i3]);
     MView b = mrow(F(th), cout);
     MView c = mview(out + size_t(r0) * d.dim_out + d.out_off[i3], n3, d.dim_out, 1, 1, n3, 0);
-    cudaError_t e = gemm_simt(int64_t(nc) * n3, cout, d.Kb[i3], a, b, c, 0, st);
+    cudaError_t e = gemm_simt(int64_t(nc) * n3, cout, d.Kb[i3], a, b, c, mode, st);
     if (e) return e;
   }
   return cudaSuccess;
@@ -127,6 +166,45 @@ int finish(cudaError_t e) {
 
 extern "C" {
 
+int tpconv_profile_enable(int on) {
+  prof().on = on != 0;
+  return TPCONV_OK;
+}
+
+int tpconv_profile_reset(void) {
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> lk(p.mu);
+  for (int i = 0; i < TPCONV_N_PHASES; ++i) {
+    for (auto& ev : p.pending[i]) {
+      cudaEventSynchronize(ev.second);
+      cudaEventDestroy(ev.first);
+      cudaEventDestroy(ev.second);
+    }
+    p.pending[i].clear();
+    p.ms[i] = 0.0;
+    p.launches[i] = 0;
+  }
+  return TPCONV_OK;
+}
+
+int tpconv_profile_read(int phase, double* ms, int64_t* launches) {
+  if (phase < 0 || phase >= TPCONV_N_PHASES) return TPCONV_ERR_INVALID_ARG;
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> lk(p.mu);
+  for (auto& ev : p.pending[phase]) {
+    float t = 0.f;
+    if (cudaEventSynchronize(ev.second) != cudaSuccess) return TPCONV_ERR_CUDA;
+    if (cudaEventElapsedTime(&t, ev.first, ev.second) != cudaSuccess) return TPCONV_ERR_CUDA;
+    p.ms[phase] += t;
+    cudaEventDestroy(ev.first);
+    cudaEventDestroy(ev.second);
+  }
+  p.pending[phase].clear();
+  if (ms) *ms = p.ms[phase];
+  if (launches) *launches = p.launches[phase];
+  return TPCONV_OK;
+}
+
 int tpconv_graph_transpose(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t* rowptr,
                            const int32_t* col, int32_t* perm, int32_t* s_rowptr, int32_t* s_recv,
                            void* workspace, size_t workspace_bytes, void* stream) {
@@ -136,21 +214,27 @@ int tpconv_graph_transpose(const tpconv_plan* plan, int64_t N, int64_t E, const 
   int st = check_ws(plan, TPCONV_OP_TRANSPOSE, N, E, workspace, workspace_bytes, &L);
   if (st) return st;
   cudaStream_t s = S(stream);
+  PhaseScope ps(TPCONV_PHASE_TRANSPOSE, s);
   char* ws = static_cast<char*>(workspace);
   int* cnt = reinterpret_cast<int*>(ws + L.off_cursor);
   int* bsum = reinterpret_cast<int*>(ws + L.off_scan);
   int* tmp = reinterpret_cast<int*>(ws + L.off_tmp);
   if (cudaMemsetAsync(cnt, 0, size_t(N + 1) * 4, s)) return TPCONV_ERR_CUDA;
-  if (E > 0) k_count_senders<<<1184, 256, 0, s>>>(E, col, cnt);
+  if (E > 0) {
+    k_count_senders<<<1184, 256, 0, s>>>(E, col, cnt);
+    note(TPCONV_PHASE_TRANSPOSE, 1);
+  }
   const int64_t n = N + 1;  // scan N+1 counts (last is 0) so s_rowptr[N] = E
   const int nb = int((n + 1023) / 1024);
   k_scan_blocks<<<nb, 1024, 0, s>>>(n, cnt, s_rowptr, bsum);
   k_scan_totals<<<1, 1024, 0, s>>>(nb, bsum, bsum + nb);
   k_scan_add<<<nb, 1024, 0, s>>>(n, s_rowptr, bsum);
+  note(TPCONV_PHASE_TRANSPOSE, 3);
   if (E > 0) {
     if (cudaMemsetAsync(cnt, 0, size_t(N + 1) * 4, s)) return TPCONV_ERR_CUDA;
     k_fill_senders<<<1184, 128, 0, s>>>(N, rowptr, col, s_rowptr, cnt, tmp);
     k_sort_segments<<<2368, 256, 0, s>>>(N, rowptr, s_rowptr, tmp, perm, s_recv);
+    note(TPCONV_PHASE_TRANSPOSE, 2);
   }
   return finish(cudaSuccess);
 }
@@ -171,9 +255,16 @@ int tpconv_forward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t*
   float* A = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_state);
   for (int64_t r0 = 0; r0 < N; r0 += L.chunk_nodes) {
     const int nc = int(std::min<int64_t>(L.chunk_nodes, N - r0));
-    if (launch_fwd_stream(d, int(r0), nc, rowptr, col, edge_vec, x, A, s)) return TPCONV_ERR_CUDA;
-    cudaError_t e = node_mix_forward(d, int(r0), nc, A, theta, out, s);
-    if (e) return TPCONV_ERR_CUDA;
+    {
+      PhaseScope ps(TPCONV_PHASE_FWD_EDGE, s);
+      if (launch_fwd_stream(d, int(r0), nc, rowptr, col, edge_vec, x, A, s)) return TPCONV_ERR_CUDA;
+      note(TPCONV_PHASE_FWD_EDGE, d.P);
+    }
+    {
+      PhaseScope ps(TPCONV_PHASE_FWD_NODE, s);
+      if (node_mix_forward(d, int(r0), nc, A, theta, out, s)) return TPCONV_ERR_CUDA;
+      note(TPCONV_PHASE_FWD_NODE, d.n_out);
+    }
   }
   return finish(cudaSuccess);
 }
@@ -201,15 +292,32 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
   if (want_edge && E > 0) {
     for (int64_t r0 = 0; r0 < N; r0 += L.chunk_nodes) {
       const int nc = int(std::min<int64_t>(L.chunk_nodes, N - r0));
-      if (node_mix_adjoint(d, int(r0), nc, g, theta, S_, s)) return TPCONV_ERR_CUDA;
-      if (launch_radj_stream(d, int(r0), nc, rowptr, col, edge_vec, x, S_, dvec, dY, db, s)) return TPCONV_ERR_CUDA;
+      {
+        PhaseScope ps(TPCONV_PHASE_BWD_NODE_G, s);
+        if (node_mix_adjoint(d, int(r0), nc, g, theta, S_, s)) return TPCONV_ERR_CUDA;
+        note(TPCONV_PHASE_BWD_NODE_G, d.n_out);
+      }
+      {
+        PhaseScope ps(TPCONV_PHASE_BWD_EDGE_R, s);
+        if (launch_radj_stream(d, int(r0), nc, rowptr, col, edge_vec, x, S_, dvec, dY, db, s))
+          return TPCONV_ERR_CUDA;
+        note(TPCONV_PHASE_BWD_EDGE_R, 1);
+      }
     }
   }
   if (want_node) {
     for (int64_t s0 = 0; s0 < N; s0 += L.chunk_nodes) {
       const int nc = int(std::min<int64_t>(L.chunk_nodes, N - s0));
-      if (launch_send_stream(d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, g, S_, s)) return TPCONV_ERR_CUDA;
-      if (node_mix_sender(d, int(s0), nc, S_, x, theta, dx, dtheta, s)) return TPCONV_ERR_CUDA;
+      {
+        PhaseScope ps(TPCONV_PHASE_BWD_EDGE_S, s);
+        if (launch_send_stream(d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, g, S_, s)) return TPCONV_ERR_CUDA;
+        note(TPCONV_PHASE_BWD_EDGE_S, d.P);
+      }
+      {
+        PhaseScope ps(TPCONV_PHASE_BWD_NODE_X, s);
+        if (node_mix_sender(d, int(s0), nc, S_, x, theta, dx, dtheta, s)) return TPCONV_ERR_CUDA;
+        note(TPCONV_PHASE_BWD_NODE_X, int64_t(d.P) * ((dx ? 1 : 0) + (dtheta ? 1 : 0)));
+      }
     }
   }
   return finish(cudaSuccess);
@@ -221,10 +329,90 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
                            const float* g, const float* gg_x, const float* gg_vec, const float* gg_theta,
                            float* d_g, float* d_x, float* d_vec, float* d_theta, void* workspace,
                            size_t workspace_bytes, void* stream) {
-  (void)plan; (void)N; (void)E; (void)rowptr; (void)col; (void)perm; (void)s_rowptr; (void)s_recv;
-  (void)edge_vec; (void)x; (void)theta; (void)g; (void)gg_x; (void)gg_vec; (void)gg_theta; (void)d_g;
-  (void)d_x; (void)d_vec; (void)d_theta; (void)workspace; (void)workspace_bytes; (void)stream;
-  return TPCONV_ERR_UNSUPPORTED;
+  if (!plan || N < 0 || E < 0) return TPCONV_ERR_INVALID_ARG;
+  if (N > 0 && (!rowptr || !x || !theta || !g)) return TPCONV_ERR_INVALID_ARG;
+  if (E > 0 && (!col || !edge_vec)) return TPCONV_ERR_INVALID_ARG;
+  const bool want_node = d_x || d_theta;
+  if (want_node && N > 0 && (!s_rowptr || (E > 0 && (!perm || !s_recv)))) return TPCONV_ERR_INVALID_ARG;
+  WsLayout L;
+  int st = check_ws(plan, TPCONV_OP_DOUBLE_BACKWARD, N, E, workspace, workspace_bytes, &L);
+  if (st) return st;
+  if ((st = ensure_device())) return st;
+  const DevPlan& d = plan->dp;
+  cudaStream_t s = S(stream);
+  const bool has_x1 = gg_x != nullptr, has_v = gg_vec != nullptr, has_t = gg_theta != nullptr;
+  if (d_theta && cudaMemsetAsync(d_theta, 0, plan->theta_numel * 4, s)) return TPCONV_ERR_CUDA;
+  if (d_x && N > 0 && cudaMemsetAsync(d_x, 0, size_t(N) * d.dim_in * 4, s)) return TPCONV_ERR_CUDA;
+  if (N == 0) return finish(cudaSuccess);
+  float* W0 = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_state);
+  const int64_t Nc = L.chunk_nodes;
+  // d_g = A1 . Theta + A0 . gg_theta
+  if (d_g) {
+    float* A1 = W0;
+    float* A0 = W0 + size_t(Nc) * plan->a_floats;
+    for (int64_t r0 = 0; r0 < N; r0 += Nc) {
+      const int nc = int(std::min<int64_t>(Nc, N - r0));
+      {
+        PhaseScope ps(TPCONV_PHASE_DBL_EDGE_A, s);
+        if (launch_dbl_a_stream(d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, A1, A0, s))
+          return TPCONV_ERR_CUDA;
+        note(TPCONV_PHASE_DBL_EDGE_A, d.P);
+      }
+      PhaseScope ps(TPCONV_PHASE_DBL_NODE_A, s);
+      if (node_mix_forward(d, int(r0), nc, A1, theta, d_g, s, 0)) return TPCONV_ERR_CUDA;
+      note(TPCONV_PHASE_DBL_NODE_A, d.n_out);
+      if (has_t) {
+        if (node_mix_forward(d, int(r0), nc, A0, gg_theta, d_g, s, 1)) return TPCONV_ERR_CUDA;
+        note(TPCONV_PHASE_DBL_NODE_A, d.n_out);
+      }
+    }
+  }
+  // d_vec from G = Theta^T g and Gt = gg_theta^T g
+  if (d_vec && E > 0) {
+    float* G = W0;
+    float* Gt = W0 + size_t(Nc) * plan->a_floats;
+    for (int64_t r0 = 0; r0 < N; r0 += Nc) {
+      const int nc = int(std::min<int64_t>(Nc, N - r0));
+      {
+        PhaseScope ps(TPCONV_PHASE_OTHER, s);
+        if (node_mix_adjoint(d, int(r0), nc, g, theta, G, s)) return TPCONV_ERR_CUDA;
+        note(TPCONV_PHASE_OTHER, d.n_out);
+        if (has_t) {
+          if (node_mix_adjoint(d, int(r0), nc, g, gg_theta, Gt, s)) return TPCONV_ERR_CUDA;
+          note(TPCONV_PHASE_OTHER, d.n_out);
+        }
+      }
+      PhaseScope ps(TPCONV_PHASE_DBL_EDGE_R, s);
+      if (launch_dbl_r_stream(d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, G, has_t ? Gt : nullptr,
+                              d_vec, s))
+        return TPCONV_ERR_CUDA;
+      note(TPCONV_PHASE_DBL_EDGE_R, 1);
+    }
+  }
+  // d_x = B1 . Theta + B0 . gg_theta ;  d_theta = x^T B1 + gg_x^T B0
+  if (want_node) {
+    float* B1 = W0;
+    float* B0 = W0 + size_t(Nc) * plan->b_floats;
+    for (int64_t s0 = 0; s0 < N; s0 += Nc) {
+      const int nc = int(std::min<int64_t>(Nc, N - s0));
+      {
+        PhaseScope ps(TPCONV_PHASE_DBL_EDGE_S, s);
+        if (launch_dbl_s_stream(d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, gg_vec, g, B1, B0, s))
+          return TPCONV_ERR_CUDA;
+        note(TPCONV_PHASE_DBL_EDGE_S, d.P);
+      }
+      PhaseScope ps(TPCONV_PHASE_DBL_NODE_X, s);
+      float* dx1 = has_v ? d_x : nullptr;
+      float* dt1 = has_v ? d_theta : nullptr;
+      if ((dx1 || dt1) && node_mix_sender(d, int(s0), nc, B1, x, theta, dx1, dt1, s)) return TPCONV_ERR_CUDA;
+      note(TPCONV_PHASE_DBL_NODE_X, int64_t(d.P) * ((dx1 ? 1 : 0) + (dt1 ? 1 : 0)));
+      float* dx0 = has_t ? d_x : nullptr;
+      float* dt0 = has_x1 ? d_theta : nullptr;
+      if ((dx0 || dt0) && node_mix_sender(d, int(s0), nc, B0, gg_x, gg_theta, dx0, dt0, s)) return TPCONV_ERR_CUDA;
+      note(TPCONV_PHASE_DBL_NODE_X, int64_t(d.P) * ((dx0 ? 1 : 0) + (dt0 ? 1 : 0)));
+    }
+  }
+  return finish(cudaSuccess);
 }
 
 }  // extern "C"

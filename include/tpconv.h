@@ -186,6 +186,35 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
                            float* d_vec, float* d_theta, void* workspace, size_t workspace_bytes,
                            void* stream);
 
+/*
+ * Diagnostics (host).  Every kernel launch of the library is counted per phase.
+ * With profiling enabled, each phase of each call is bracketed by CUDA events
+ * recorded on the call's stream; tpconv_profile_read synchronises those events
+ * and returns the summed device time of a phase.  Profiling state is process-
+ * wide and not thread-safe; it does not change results.
+ */
+#define TPCONV_PHASE_TRANSPOSE 0   /* sender-sorted view of the graph          */
+#define TPCONV_PHASE_FWD_EDGE 1    /* forward receiver edge stream -> A        */
+#define TPCONV_PHASE_FWD_NODE 2    /* out = A . Theta                          */
+#define TPCONV_PHASE_BWD_NODE_G 3  /* G = g . Theta^T                          */
+#define TPCONV_PHASE_BWD_EDGE_R 4  /* receiver adjoint stream -> dvec, dY, db  */
+#define TPCONV_PHASE_BWD_EDGE_S 5  /* sender stream -> B                       */
+#define TPCONV_PHASE_BWD_NODE_X 6  /* dx = B . Theta, dtheta = x^T B           */
+#define TPCONV_PHASE_DBL_EDGE_A 7  /* double backward receiver stream -> A0,A1 */
+#define TPCONV_PHASE_DBL_NODE_A 8  /* d_g = A1 . Theta + A0 . gg_theta         */
+#define TPCONV_PHASE_DBL_EDGE_R 9  /* double backward adjoint stream -> d_vec  */
+#define TPCONV_PHASE_DBL_EDGE_S 10 /* double backward sender stream -> B0, B1  */
+#define TPCONV_PHASE_DBL_NODE_X 11 /* d_x, d_theta                             */
+#define TPCONV_PHASE_OTHER 12      /* memsets, packing, G for double backward  */
+#define TPCONV_N_PHASES 13
+
+int tpconv_profile_enable(int on);  /* 1: record events from now on; 0: stop    */
+int tpconv_profile_reset(void);     /* drop recorded events and launch counts   */
+/* ms: summed device milliseconds of the phase since the last reset (needs
+ * profiling enabled while the calls ran); launches: kernels launched in the
+ * phase since the last reset (always counted).  Either pointer may be NULL. */
+int tpconv_profile_read(int phase, double* ms, int64_t* launches);
+
 #ifdef __cplusplus
 }
 #endif

@@ -167,3 +167,35 @@ def test_mace_full_size_sampled(T):
     Y2, b2 = conv.geometry(prob, vec[sm])
     dx, _, _, _ = conv.backward_core(prob, N, col[sm].astype(np.int64), recv[sm], x, Y2, b2, th, g)
     assert rel(bw["dx"][ss], dx[ss]) < TOL_FP32
+
+
+DBL_CASES = {
+    "tiny_all": ("tiny", ("x", "v", "t")),
+    "mixed_all": ("mixed_l3", ("x", "v", "t")),
+    "mixed_force_shape": ("mixed_l3", ("x", "v")),
+    "radius_only_vec": ("radius_small", ("v",)),
+    "wide_only_theta_x": ("wide_channels", ("x", "t")),
+}
+
+
+@pytest.mark.parametrize("case", list(DBL_CASES))
+def test_double_backward_parity(T, case):
+    import torch
+    base, which = DBL_CASES[case]
+    irr_in, lsh, irr_out, R, rad, rp, gf = CASES[base]
+    plan, prob, G, inp = make(T, irr_in, lsh, irr_out, R, rad, rp, gf(), seed=51)
+    rowptr, col, vec, x, th, g = inp
+    r32 = lambda a: a.astype(np.float32).astype(np.float64)
+    ggx = r32(W.normal(x.shape, 52)) if "x" in which else None
+    ggv = r32(W.normal(vec.shape, 53)) if "v" in which else None
+    ggt = r32(W.normal(th.shape, 54) * 0.05) if "t" in which else None
+    d = lambda a: None if a is None else dev(a, torch.float32)
+    out = T.double_backward(plan, G, d(x), d(th), d(g), d(ggx), d(ggv), d(ggt))
+    torch.cuda.synchronize()
+    ref = conv.double_backward(prob, rowptr, col, vec, x, th, g, ggx, ggv, ggt)
+    for k in ("d_g", "d_x", "d_vec", "d_theta"):
+        got = out[k].cpu().numpy()
+        if np.abs(ref[k]).max() == 0:
+            assert np.abs(got).max() == 0, k
+        else:
+            assert rel(got, ref[k]) < TOL_FP32, (k, rel(got, ref[k]))
