@@ -1,0 +1,402 @@
+#!/usr/bin/env python3
+"""Benchmark of the streaming CG tensor-product convolution on B200.
+
+One step = one pass of the whole hot path over one synthetic batch of the
+mace-like layer (4096 atoms in a periodic box at 0.1 atoms/A^3, all pairs within
+5 A, 64x0e+64x1o+64x2e -> same, SH l<=3, R=8 Bessel radial basis): sender-sorted
+graph view, forward, backward (dx, dTheta, dvec) and double backward in the
+force-training shape (gg_x, gg_vec given, gg_Theta = 0) -> d_g, d_x, d_vec,
+d_Theta.  The headline value is edges per second of that step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torch.distributed.run: every rank processes its own graph
+(seed = rank) with no collective on the data path (weak scaling); the step time
+is the max over ranks.  --impl reference times the CPU oracle on a bounded
+sample of the same workload (the pages ship no runnable reference).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+WORKLOAD = ("mace-like layer: 4096 atoms, periodic cube at 0.1 atoms/A^3, 5 A radius graph, "
+            "64x0e+64x1o+64x2e -> 64x0e+64x1o+64x2e, SH l<=3, R=8 Bessel")
+METRIC = "edges/s (fwd + bwd + double bwd step)"
+L2_BYTES = 126 * 1024 * 1024
+FP32_LANES_PER_SM = 128
+N_SM = 148
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="mace")
+    ap.add_argument("--gemm", default="fp32", choices=["fp32", "tf32", "simt"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "sm_max_mhz": 1965.0}, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work model (per edge), from the plan's path table and CG pattern
+# ---------------------------------------------------------------------------
+def work_model(T, plan):
+    R = plan.R
+    nnz_cache = {}
+    fw = bw_r = bw_s = db_a = db_r = db_s = 0
+    for p in plan.paths:
+        key = (p["l1"], p["l2"], p["l3"])
+        if key not in nnz_cache:
+            C = T.tpconv_cg_coefficients(*key)
+            nz = np.abs(C) > 0
+            nnz_cache[key] = (int(nz.sum()), int(nz.any(axis=1).sum()))
+        nnz, mnz = nnz_cache[key]
+        n1, n3 = 2 * p["l1"] + 1, 2 * p["l3"] + 1
+        ci, co = p["c_in"], p["c_out"]
+        fw += nnz + ci * (mnz + R * n3)                           # M_e, M x, b (x) T
+        bw_r += nnz + ci * (mnz + 2 * R * n3 + mnz + nnz)         # M x, dT, db, C(x, dT)
+        bw_s += nnz + co * (mnz + R * n1)                         # M_e, M^T g, b (x) U
+        db_a += 2 * nnz + ci * (3 * mnz + 3 * R * n3)
+        db_r += 2 * nnz + ci * (3 * mnz + 6 * R * n3 + 3 * (mnz + nnz))
+        db_s += 2 * nnz + co * (2 * mnz + 3 * R * n1)
+    return {"fwd_edge": fw, "bwd_edge_r": bw_r, "bwd_edge_s": bw_s, "dbl_edge_a": db_a, "dbl_edge_r": db_r,
+            "dbl_edge_s": db_s}
+
+
+def gemm_flops(plan_info, N):
+    """Node-level Theta contractions per step (FMAs): out, G, dx, dTheta, d_g, d_x, d_Theta."""
+    per = plan_info["mix_fma_per_node"]
+    return {"fwd_node": per * N, "bwd_node_g": per * N, "bwd_node_x": 2 * per * N, "dbl_node_a": per * N,
+            "dbl_node_x": 2 * per * N}
+
+
+class ClockSampler:
+    def __init__(self, index, path):
+        self.path = path
+        self.proc = None
+        self.index = index
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        try:
+            rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
+        except OSError:
+            rows = []
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows]
+        mx = [float(r[2]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        n = 1
+    return int(n)
+
+
+def oracle_sample(cfg, graph, n_recv, seed=100):
+    """Oracle step (fwd + bwd + double bwd) on the edges of the first n_recv receivers."""
+    from oracle import conv
+    c = W.CONFIGS[cfg]
+    prob = conv.Problem(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], c["radial"],
+                        tuple(c["radial_params"]))
+    rowptr, col, vec = graph
+    N = len(rowptr) - 1
+    e1 = int(rowptr[n_recv])
+    rp = np.asarray(rowptr[:n_recv + 1], dtype=np.int64)
+    x = W.normal((N, prob.dim_in), seed)
+    th = W.theta([(prob.R * p.c_in * p.c_out, 1 / np.sqrt(prob.R * p.c_in)) for p in prob.paths], seed + 1)
+    g = np.zeros((n_recv, prob.dim_out))
+    g[:] = W.normal((n_recv, prob.dim_out), seed + 2)
+    ggx = W.normal((N, prob.dim_in), seed + 3)
+    ggv = W.normal((e1, 3), seed + 4)
+
+    def step():
+        send = np.asarray(col[:e1], dtype=np.int64)
+        recv = conv.receivers_of(rp)
+        Y, b = conv.geometry(prob, vec[:e1])
+        conv.forward_core(prob, n_recv, send, recv, x, Y, b, th)
+        conv.backward(prob, rp, col[:e1], vec[:e1], x, th, g)
+        conv.double_backward(prob, rp, col[:e1], vec[:e1], x, th, g, ggx, ggv, None)
+
+    return step, e1
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    graph = W.graph_for(args.config, 0)
+    n_recv = 8
+    step, e = oracle_sample(args.config, graph, n_recv)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    v = e / dt
+    cores = cpu_cores()
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "edges/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": f"edges of the first {n_recv} receivers ({e} edges)"},
+            "cpu_baseline": {"value": v, "unit": "edges/s", "cores": cores, "kind": "oracle",
+                             "sample": f"fp64 numpy oracle, conventional schedule, {e} edges per step"},
+            "e2e": {"value": v, "unit": "edges/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+
+    import equivariant_gnn_tensor_receiver_b200 as T
+    from equivariant_gnn_tensor_receiver_b200 import _lib as L
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    c = W.CONFIGS[args.config]
+    rowptr, col, vec = W.graph_for(args.config, rank)
+    N, E = len(rowptr) - 1, len(col)
+    plan = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], radial=c["radial"],
+                  radial_params=c["radial_params"], gemm=args.gemm)
+    f32 = torch.float32
+    pin = lambda a, dt=f32: torch.as_tensor(np.ascontiguousarray(a), dtype=dt).pin_memory()
+    host = {
+        "rowptr": pin(rowptr, torch.int32), "col": pin(col, torch.int32), "vec": pin(vec),
+        "x": pin(W.normal((N, plan.dim_in), 10 + rank)),
+        "theta": pin(W.theta([(plan.R * p["c_in"] * p["c_out"], 1 / np.sqrt(plan.R * p["c_in"]))
+                              for p in plan.paths], 11 + rank)),
+        "g": pin(W.normal((N, plan.dim_out), 12 + rank)),
+        "gg_x": pin(W.normal((N, plan.dim_in), 13 + rank)),
+        "gg_vec": pin(W.normal((E, 3), 14 + rank)),
+    }
+    d = {k: v.to(dev) for k, v in host.items()}
+    outs = {
+        "out": torch.empty(N, plan.dim_out, device=dev), "dx": torch.empty(N, plan.dim_in, device=dev),
+        "dtheta": torch.empty(plan.theta_numel, device=dev), "dvec": torch.empty(E, 3, device=dev),
+        "d_g": torch.empty(N, plan.dim_out, device=dev), "d_x": torch.empty(N, plan.dim_in, device=dev),
+        "d_vec": torch.empty(E, 3, device=dev), "d_theta": torch.empty(plan.theta_numel, device=dev),
+    }
+    hout = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in outs.items()}
+    perm = torch.empty(E, dtype=torch.int32, device=dev)
+    s_rowptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    s_recv = torch.empty(E, dtype=torch.int32, device=dev)
+    ws = {op: T.workspace(plan, op, N, E, dev) for op in (L.OP_FORWARD, L.OP_BACKWARD, L.OP_DOUBLE_BACKWARD,
+                                                          L.OP_TRANSPOSE)}
+    ws_bytes = sum(w.numel() for w in ws.values())
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(src):
+        L.tpconv_graph_transpose(plan, N, E, src["rowptr"], src["col"], perm, s_rowptr, s_recv, ws[L.OP_TRANSPOSE])
+        L.tpconv_forward(plan, N, E, src["rowptr"], src["col"], src["vec"], src["x"], src["theta"], outs["out"],
+                         ws[L.OP_FORWARD])
+        L.tpconv_backward(plan, N, E, src["rowptr"], src["col"], perm, s_rowptr, s_recv, src["vec"], src["x"],
+                          src["theta"], src["g"], outs["dx"], outs["dtheta"], outs["dvec"], None, None,
+                          ws[L.OP_BACKWARD])
+        L.tpconv_double_backward(plan, N, E, src["rowptr"], src["col"], perm, s_rowptr, s_recv, src["vec"],
+                                 src["x"], src["theta"], src["g"], src["gg_x"], src["gg_vec"], None, outs["d_g"],
+                                 outs["d_x"], outs["d_vec"], outs["d_theta"], ws[L.OP_DOUBLE_BACKWARD])
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def allmax(v):
+        if world == 1:
+            return v
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def allsum(v):
+        if world == 1:
+            return v
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+
+    for _ in range(max(args.warmup, 3)):
+        step(d)
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats(dev)
+    base_alloc = torch.cuda.memory_allocated(dev)
+    L.tpconv_profile_reset()
+    L.tpconv_profile_enable(True)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clk_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv") if os.path.isdir(
+        os.path.join(ROOT, "gpurun_out")) else f"/tmp/tpconv_clocks_{rank}.csv"
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index, clk_path) as clk:
+        time.sleep(0.3)
+        for i in range(args.steps):
+            flush.zero_()
+            evs[i][0].record()
+            step(d)
+            evs[i][1].record()
+        torch.cuda.synchronize()
+    barrier()
+    L.tpconv_profile_enable(False)
+    step_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    step_ms_max = allmax(step_ms)
+    E_total = allsum(E)
+    peak_mem = torch.cuda.max_memory_allocated(dev)
+    prof = L.profile_all()
+    launches = int(sum(n for _, n in prof.values()))
+
+    # end to end: inputs from pinned host memory, all outputs back to pinned host memory
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(v.numel() * v.element_size() for v in outs.values())
+    e2e = []
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for k, v in host.items():
+            d[k].copy_(v, non_blocking=True)
+        step(d)
+        for k, v in outs.items():
+            hout[k].copy_(v, non_blocking=True)
+        b.record()
+        b.synchronize()
+        e2e.append(a.elapsed_time(b))
+    e2e_ms = allmax(sum(e2e) / len(e2e))
+
+    # roofline of the dominant phase
+    peaks, peak_src = measured_peaks()
+    wm = work_model(T, plan)
+    phase_ms = {k: ms / args.steps for k, (ms, _) in prof.items()}
+    dom = max(phase_ms, key=lambda k: phase_ms[k])
+    roof = {"phase": dom, "bound": None, "achieved": None, "peak": None, "unit": None, "frac": None,
+            "traffic": None}
+    sm_max = peaks.get("sm_max_mhz", 1965.0)
+    if dom in wm:
+        flops = 2.0 * wm[dom] * E
+        ach = flops / (phase_ms[dom] * 1e-3) / 1e12
+        peak = N_SM * FP32_LANES_PER_SM * 2 * sm_max * 1e6 / 1e12
+        roof.update(bound="alu", achieved=ach, peak=peak, unit="TFLOP/s", frac=ach / peak,
+                    peak_source=f"148 SM x 128 FP32 lanes x 2 x {sm_max:.0f} MHz (max clock, {peak_src} file)",
+                    work=f"{wm[dom]} algorithmic FMA per edge x {E} edges")
+    try:
+        with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+            tr = json.load(f).get(dom)
+        if tr and tr.get("lib_mtime") == int(os.path.getmtime(L.LIB_PATH)):
+            roof["traffic"] = tr["bytes_per_step"]
+    except (OSError, ValueError):
+        pass
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        stepc, ec = oracle_sample(args.config, (rowptr, col, vec), 4)
+        stepc()
+        t0 = time.perf_counter()
+        reps = 0
+        while time.perf_counter() - t0 < 10.0 or reps < 1:
+            stepc()
+            reps += 1
+        dt = (time.perf_counter() - t0) / reps
+        cpu = {"value": ec / dt, "unit": "edges/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"fp64 numpy oracle step (fwd+bwd+double bwd) on the {ec} edges of 4 receivers, "
+                         f"{reps} reps"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": E_total / (step_ms_max * 1e-3), "unit": "edges/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": step_ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "nodes_per_gpu": N, "edges_per_gpu": E, "gemm": args.gemm,
+                       "step": "graph transpose + fwd + bwd(dx,dTheta,dvec) + double bwd(gg_x,gg_vec)",
+                       "l2": "256 MiB buffer zeroed before every timed step, outside the events",
+                       "parallelism": f"{world} independent replicas (one graph per rank)"},
+            "e2e": {"value": E_total / (e2e_ms * 1e-3), "unit": "edges/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "clocks": clk.summary(),
+            "phases_ms": {k: round(v, 4) for k, v in phase_ms.items() if v > 0},
+            "peak_mem_bytes": peak_mem, "workspace_bytes": ws_bytes, "resident_bytes_before_step": base_alloc,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

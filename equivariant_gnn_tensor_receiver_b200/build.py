@@ -22,8 +22,6 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libtpconv.so")
 
-CU_SOURCES = ["tpconv.cu", "stream_fwd.cu", "stream_send.cu", "stream_radj.cu", "stream_dbl.cu",
-              "gemm_tc.cu"]
 CXX_SOURCES = ["plan.cpp"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -32,25 +30,36 @@ NVCC_FLAGS = ARCH + ["-lineinfo", "-O3", "-std=c++17", "--expt-relaxed-constexpr
 CXX_FLAGS = ["-O2", "-fPIC", "-std=c++17", f"-I{os.path.join(ROOT, 'include')}"]
 
 
-def _headers_mtime():
-    m = 0.0
-    for d in (CSRC, os.path.join(ROOT, "include")):
-        for f in os.listdir(d):
-            if f.endswith((".h", ".cuh")):
-                m = max(m, os.path.getmtime(os.path.join(d, f)))
+def _cu_sources():
+    return sorted(f for f in os.listdir(CSRC) if f.endswith(".cu"))
+
+
+def _deps_mtime(dep_file, src_path):
+    """Newest mtime among the source and the headers listed in its -MD file."""
+    m = os.path.getmtime(src_path)
+    try:
+        text = open(dep_file).read().replace("\\\n", " ")
+    except OSError:
+        return None
+    for tok in text.split(":", 1)[-1].split():
+        if os.path.exists(tok):
+            m = max(m, os.path.getmtime(tok))
     return m
 
 
-def _compile(src, force, hdr):
+def _compile(src, force, _unused=None):
     path = os.path.join(CSRC, src)
     obj = os.path.join(BUILD, src + ".o")
     log = os.path.join(BUILD, src + ".log")
-    if not force and os.path.exists(obj) and os.path.getmtime(obj) >= max(os.path.getmtime(path), hdr):
-        return obj, None
+    dep = os.path.join(BUILD, src + ".d")
+    if not force and os.path.exists(obj):
+        newest = _deps_mtime(dep, path)
+        if newest is not None and os.path.getmtime(obj) >= newest:
+            return obj, None
     if src.endswith(".cu"):
-        cmd = [NVCC] + NVCC_FLAGS + ["-c", path, "-o", obj]
+        cmd = [NVCC] + NVCC_FLAGS + ["-MD", "-MF", dep, "-c", path, "-o", obj]
     else:
-        cmd = [os.environ.get("CXX", "g++")] + CXX_FLAGS + ["-c", path, "-o", obj]
+        cmd = [os.environ.get("CXX", "g++")] + CXX_FLAGS + ["-MD", "-MF", dep, "-c", path, "-o", obj]
     res = subprocess.run(cmd, capture_output=True, text=True)
     with open(log, "w") as f:
         f.write(" ".join(cmd) + "\n" + res.stdout + res.stderr)
@@ -61,19 +70,25 @@ def _compile(src, force, hdr):
 
 def build(force: bool = False, verbose: bool = True) -> str:
     os.makedirs(BUILD, exist_ok=True)
-    hdr = _headers_mtime()
-    sources = [s for s in CXX_SOURCES + CU_SOURCES if os.path.exists(os.path.join(CSRC, s))]
-    with cf.ThreadPoolExecutor(max_workers=len(sources)) as ex:
-        results = list(ex.map(lambda s: _compile(s, force, hdr), sources))
+    sources = CXX_SOURCES + _cu_sources()
+    # heaviest units first so the pool stays busy
+    sources.sort(key=lambda s: (0 if ("dbl_r" in s or "radj" in s) else 1, s))
+    with cf.ThreadPoolExecutor(max_workers=min(len(sources), os.cpu_count() or 8)) as ex:
+        results = list(ex.map(lambda s: _compile(s, force), sources))
     errs = [e for _, e in results if e]
     if errs:
         raise RuntimeError("\n".join(errs))
     objs = [o for o, _ in results]
+    stale = [f for f in os.listdir(BUILD) if f.endswith(".cu.o") and f[:-2] not in _cu_sources()]
+    for f in stale:
+        os.remove(os.path.join(BUILD, f))
     if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        cmd = [NVCC] + ARCH + ["-shared", "-cudart", "static", "-o", LIB] + objs
+        tmp = LIB + ".tmp"
+        cmd = [NVCC] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
             raise RuntimeError("link failed:\n" + res.stderr[-4000:])
+        os.replace(tmp, LIB)  # atomic: a concurrent reader sees the old or the new library
     if verbose:
         print(f"built {LIB}")
     return LIB

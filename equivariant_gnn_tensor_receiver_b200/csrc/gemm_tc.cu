@@ -1,0 +1,434 @@
+// Tensor-core GEMM for the node-level Theta contraction (sm_100a: tcgen05 + TMEM + TMA).
+//
+//   C[m, n] (+)= sum_k A[m, k] B[n, k]       A: [M][K] fp32 row-major (K-major)
+//                                            B: [N][K] fp32 row-major (K-major)
+// C is written through a strided view, so rows (node, m) and columns (channel)
+// land directly in the [node][mul][2l+1] feature layout.
+//
+// This is the mixing step of the streaming schedule ("Sobek", arXiv 2607.18074,
+// abstract: fully connected multiplicity mixing applied to bounded receiver-side
+// state): out_blk = A_blk . Theta_blk with A the receiver-side state.
+//
+// Precision modes:
+//   TF32   one kind::tf32 MMA per K step (operands read as TF32).
+//   3xTF32 fp32-accurate split (Ootomo & Yokota, 2022): a_hi = rn_tf32(a),
+//          a_lo = rn_tf32(a - a_hi), both exactly representable in TF32;
+//          C += A_hi B_hi + A_hi B_lo + A_lo B_hi.  Round-to-nearest (not
+//          truncation) keeps the neglected terms uncorrelated with the sign of
+//          a*b, so their sum grows like sqrt(K), not K.  The B split is
+//          precomputed; the A split is done in shared memory by four converter
+//          warps between the TMA load and the MMA.
+//
+// CTA: 6 warps.  warp 0 issues TMA loads (128 x 32 A tile and BN x 32 B tile,
+// 128-byte swizzle) into a ring of shared-memory stages; warp 1 owns the TMEM
+// accumulator (128 lanes x BN fp32 columns) and issues the MMAs from one thread;
+// warps 2-5 split A (3xTF32) and run the epilogue (tcgen05.ld -> global).
+// Every wait is bounded; on expiry the kernel records an error code, stops
+// issuing work, waits (bounded) for its own loads, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "gemm_tc.h"
+
+namespace tpc {
+
+__device__ int g_tc_error;  // first error code recorded by a tensor-core GEMM (0 = none)
+
+namespace {
+
+constexpr int kBM = 128, kBK = 32;  // rows per CTA, fp32 K per stage (128 bytes)
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits give up after 2 s
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// bounded wait; returns false (and records `code`) when the limit expires
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, int code) {
+  if (mbar_try(b, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try(b, parity)) {
+    if (global_ns() - t0 > kWaitLimitNs) {
+      atomicCAS(&g_tc_error, 0, code);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ float rn_tf32(float a) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(a));
+  return __uint_as_float(r);
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// K-major, 128-byte swizzle shared-memory matrix descriptor (sm_100 layout):
+// start address >> 4 in [0,14), leading byte offset (unused here) in [16,30),
+// stride byte offset 1024 (8 rows x 128 B) >> 4 in [32,46), version 1 at [46,48),
+// layout type SWIZZLE_128B = 2 at [61,64).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr & 0x3FFFF) >> 4);
+  d |= uint64_t(1) << 16;
+  d |= uint64_t(1024 >> 4) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(2) << 61;
+  return d;
+}
+
+// instruction descriptor of kind::tf32, fp32 accumulate, both operands K-major
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
+  return (1u << 4)                 // D format F32
+         | (2u << 7) | (2u << 10)  // A, B format TF32
+         | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+template <int BN>
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int BN>
+struct TcSmem {
+  static constexpr int kA = kBM * kBK * 4;   // 16 KB
+  static constexpr int kB = BN * kBK * 4;    // BN x 128 B
+  static constexpr int kStage = 2 * kA + 2 * kB;
+  static constexpr int kStages = (200 * 1024) / kStage >= 4 ? 4 : ((200 * 1024) / kStage >= 3 ? 3 : 2);
+  static constexpr int kBytes = kStages * kStage + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+template <int BN, bool SPLIT>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmBlo, int M, int N, int K, TcOut out, int accumulate) {
+  using SM = TcSmem<BN>;
+  constexpr int S = SM::kStages;
+  constexpr uint32_t kCols = BN < 32 ? 32 : BN;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + S * SM::kStage);
+  uint64_t* conv = full + S;
+  uint64_t* empty = conv + S;
+  uint64_t* accf = empty + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kBM;
+  const int n0 = blockIdx.y * BN;
+  const int nk = (K + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&conv[s], 128);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;");
+  const uint32_t tmem = *tmem_slot;
+
+  auto sA = [&](int s) { return base + s * SM::kStage; };
+  auto sAlo = [&](int s) { return base + s * SM::kStage + SM::kA; };
+  auto sB = [&](int s) { return base + s * SM::kStage + 2 * SM::kA; };
+  auto sBlo = [&](int s) { return base + s * SM::kStage + 2 * SM::kA + SM::kB; };
+
+  int issued = 0;  // TMA stages issued by warp 0
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t bytes = SM::kA + (SPLIT ? 2 : 1) * SM::kB;
+      for (int kt = 0; kt < nk; ++kt) {
+        const int s = kt % S;
+        if (kt >= S && !mbar_wait(&empty[s], ((kt / S) + 1) & 1, 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        if (*abort_flag) break;
+        mbar_expect_tx(&full[s], bytes);
+        tma_load_2d(sA(s), &tmA, &full[s], kt * kBK, m0);
+        tma_load_2d(sB(s), &tmB, &full[s], kt * kBK, n0);
+        if (SPLIT) tma_load_2d(sBlo(s), &tmBlo, &full[s], kt * kBK, n0);
+        issued = kt + 1;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_tf32(kBM, BN);
+      for (int kt = 0; kt < nk; ++kt) {
+        const int s = kt % S;
+        const uint32_t par = (kt / S) & 1;
+        if (!mbar_wait(SPLIT ? &conv[s] : &full[s], par, 2) || *abort_flag) {
+          *abort_flag = 1;
+          break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;");
+        const uint32_t a = smem_u32(sA(s)), al = smem_u32(sAlo(s)), b = smem_u32(sB(s)), bl = smem_u32(sBlo(s));
+#pragma unroll
+        for (int kk = 0; kk < kBK / 8; ++kk) {
+          const uint32_t off = kk * 32;  // 8 TF32 = 32 bytes along K inside the swizzle atom
+          const uint32_t acc = (kt > 0 || kk > 0) ? 1u : 0u;
+          mma_tf32(tmem, sw128_desc(a + off), sw128_desc(b + off), idesc, acc);
+          if (SPLIT) {
+            mma_tf32(tmem, sw128_desc(a + off), sw128_desc(bl + off), idesc, 1u);
+            mma_tf32(tmem, sw128_desc(al + off), sw128_desc(b + off), idesc, 1u);
+          }
+        }
+        mma_commit(&empty[s]);
+      }
+      mma_commit(accf);
+    }
+  } else {
+    // warps 2..5: split A in shared memory (3xTF32), then the epilogue
+    const int t = threadIdx.x - 64;  // 0..127
+    if (SPLIT) {
+      for (int kt = 0; kt < nk; ++kt) {
+        const int s = kt % S;
+        if (!mbar_wait(&full[s], (kt / S) & 1, 3) || *abort_flag) {
+          *abort_flag = 1;
+          break;
+        }
+        float4* a4 = reinterpret_cast<float4*>(sA(s));
+        float4* l4 = reinterpret_cast<float4*>(sAlo(s));
+#pragma unroll 4
+        for (int i = t; i < kBM * kBK / 4; i += 128) {
+          float4 v = a4[i], h, l;
+          h.x = rn_tf32(v.x);
+          h.y = rn_tf32(v.y);
+          h.z = rn_tf32(v.z);
+          h.w = rn_tf32(v.w);
+          l.x = rn_tf32(v.x - h.x);
+          l.y = rn_tf32(v.y - h.y);
+          l.z = rn_tf32(v.z - h.z);
+          l.w = rn_tf32(v.w - h.w);
+          a4[i] = h;
+          l4[i] = l;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(&conv[s]);
+      }
+    }
+    const bool ok = mbar_wait(accf, 0, 4) && !*abort_flag;
+    asm volatile("tcgen05.fence::after_thread_sync;");
+    if (ok) {
+      const int q = warp & 3;  // TMEM lane quadrant this warp may access
+      const int row = m0 + q * 32 + lane;
+      const int64_t rbase = (row / out.rdiv) * out.r_hi + (row % out.rdiv) * out.r_lo;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 16) {
+        float v[16];
+        tmem_ld16<BN>(tmem + (uint32_t(q * 32) << 16) + uint32_t(c), v);
+        if (row < M) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int col = n0 + c + i;
+            if (col < N) {
+              float* dst = out.p + rbase + int64_t(col) * out.c_hi;
+              *dst = accumulate ? *dst + v[i] : v[i];
+            }
+          }
+        }
+      }
+    }
+  }
+  // drain: the producer waits (bounded) for the loads it issued so no copy is
+  // in flight when the CTA exits, then TMEM is released
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    for (int kt = (issued > S ? issued - S : 0); kt < issued; ++kt) mbar_wait(&full[kt % S], (kt / S) & 1, 5);
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;");
+  __syncthreads();
+  if (warp == 1) {
+    asm volatile("tcgen05.fence::after_thread_sync;");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols));
+  }
+}
+
+// ---- host side ---------------------------------------------------------------
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encoder() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  });
+  return fn;
+}
+
+// rows x cols fp32 row-major with leading dimension ld (elements); box box_rows x 32
+bool make_map(CUtensorMap* m, const float* p, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
+  EncodeFn enc = encoder();
+  if (!enc) return false;
+  if ((reinterpret_cast<uintptr_t>(p) & 15) || ((ld * 4) & 15) || rows <= 0 || cols <= 0) return false;
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(ld * 4)};
+  cuuint32_t box[2] = {cuuint32_t(kBK), cuuint32_t(box_rows)};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(p), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, bool SPLIT>
+cudaError_t run(const float* A, int64_t lda, const float* B, const float* Blo, int64_t ldb, int M, int N, int K,
+                TcOut out, int accumulate, cudaStream_t st) {
+  CUtensorMap ta, tb, tbl;
+  if (!make_map(&ta, A, M, K, lda, kBM) || !make_map(&tb, B, N, K, ldb, BN)) return cudaErrorInvalidValue;
+  if (SPLIT && !make_map(&tbl, Blo, N, K, ldb, BN)) return cudaErrorInvalidValue;
+  if (!SPLIT) tbl = tb;
+  using SM = TcSmem<BN>;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SM::kBytes);
+    if (e) return e;
+    attr_done[dev] = true;
+  }
+  dim3 grid(unsigned((M + kBM - 1) / kBM), unsigned((N + BN - 1) / BN));
+  k_gemm_tc<BN, SPLIT><<<grid, 192, SM::kBytes, st>>>(ta, tb, tbl, M, N, K, out, accumulate);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gemm_tc_supported(const float* A, int64_t lda, const float* B, int64_t ldb, int M, int N, int K) {
+  if (!encoder()) return false;
+  if (M <= 0 || N <= 0 || K <= 0) return false;
+  if ((reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(B) & 15)) return false;
+  if ((lda & 3) || (ldb & 3)) return false;
+  return true;
+}
+
+cudaError_t gemm_tc(const float* A, int64_t lda, const float* B, const float* Blo, int64_t ldb, int M, int N, int K,
+                    TcOut out, int accumulate, bool split, cudaStream_t st) {
+  const int bn = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256));
+  if (split) {
+    switch (bn) {
+      case 32: return run<32, true>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
+      case 64: return run<64, true>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
+      case 128: return run<128, true>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
+      default: return run<256, true>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
+    }
+  }
+  switch (bn) {
+    case 32: return run<32, false>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
+    case 64: return run<64, false>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
+    case 128: return run<128, false>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
+    default: return run<256, false>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
+  }
+}
+
+cudaError_t gemm_tc_read_error(int* code, cudaStream_t st) {
+  int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(code, g_tc_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st);
+  if (e) return e;
+  if ((e = cudaStreamSynchronize(st))) return e;
+  return cudaMemcpyToSymbolAsync(g_tc_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+}
+
+// Theta^T split: hi[n][k] = rn_tf32(Theta[k][n]), lo = rn_tf32(Theta - hi)
+__global__ void k_split_transpose(const float* __restrict__ th, int K, int N, float* __restrict__ hi,
+                                  float* __restrict__ lo) {
+  __shared__ float tile[32][33];
+  const int k0 = blockIdx.x * 32, n0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int k = k0 + i, n = n0 + threadIdx.x;
+    tile[i][threadIdx.x] = (k < K && n < N) ? th[int64_t(k) * N + n] : 0.f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int n = n0 + i, k = k0 + threadIdx.x;
+    if (n < N && k < K) {
+      const float v = tile[threadIdx.x][i];
+      const float h = rn_tf32(v);
+      if (lo) {
+        hi[int64_t(n) * K + k] = h;
+        lo[int64_t(n) * K + k] = rn_tf32(v - h);
+      } else {
+        hi[int64_t(n) * K + k] = v;
+      }
+    }
+  }
+}
+
+cudaError_t split_transpose(const float* th, int K, int N, float* hi, float* lo, cudaStream_t st) {
+  dim3 grid(unsigned((K + 31) / 32), unsigned((N + 31) / 32));
+  k_split_transpose<<<grid, dim3(32, 8), 0, st>>>(th, K, N, hi, lo);
+  return cudaGetLastError();
+}
+
+}  // namespace tpc

@@ -1,0 +1,28 @@
+// Tensor-core (tcgen05) GEMM for the node-level Theta contraction.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tpc {
+
+// C(i, j) = p[(i / rdiv) * r_hi + (i % rdiv) * r_lo + j * c_hi]
+struct TcOut {
+  float* p;
+  int64_t rdiv, r_hi, r_lo, c_hi;
+};
+
+// TMA / descriptor requirements: 16-byte aligned bases, row pitches a multiple of 4 floats.
+bool gemm_tc_supported(const float* A, int64_t lda, const float* B, int64_t ldb, int M, int N, int K);
+
+// C (+)= A[M][K] . B[N][K]^T.  split = 3xTF32 (B and Blo precomputed), else one TF32 pass.
+cudaError_t gemm_tc(const float* A, int64_t lda, const float* B, const float* Blo, int64_t ldb, int M, int N, int K,
+                    TcOut out, int accumulate, bool split, cudaStream_t st);
+
+// Theta block [K][N] -> hi = its transpose [N][K] (rounded to TF32 when lo != null), lo = remainder.
+cudaError_t split_transpose(const float* th, int K, int N, float* hi, float* lo, cudaStream_t st);
+
+// First error recorded by a bounded wait inside a tensor-core GEMM (0 = none); clears it. Synchronises st.
+cudaError_t gemm_tc_read_error(int* code, cudaStream_t st);
+
+}  // namespace tpc

@@ -345,7 +345,64 @@ int tpconv_plan_create(tpconv_plan** out, const char* irreps_in, int l_sh_max,
   }
   d.sm_floats = sm;
   d.sm_floats2 = sm2;
-  if (size_t(std::max(sm, sm2)) * 4 > 227 * 1024) {
+  // fused streams: all paths of a node in one CTA (one warp per path, passes of <= 14 warps)
+  {
+    const int passes = (P + 13) / 14;
+    d.fz_warps = std::max(1, (P + passes - 1) / passes);
+    int msz = 0;
+    for (int i = 0; i < P; ++i) {
+      d.path[i].smf_off = msz;
+      msz += kEdgeBatch * ((d.path[i].nmz + 3) & ~3);
+    }
+    d.fz_cpl_f = d.max_c_in > 32 ? 2 : 1;
+    d.fz_cpl_s = d.max_c_out > 32 ? 2 : 1;
+    d.fz_xw_f = 0;
+    for (int i = 0; i < d.n_in; ++i) d.fz_xw_f += std::min(32 * d.fz_cpl_f, d.in_mul[i]) * (2 * d.in_l[i] + 1);
+    d.fz_xw_s = 0;
+    for (int i = 0; i < d.n_out; ++i) d.fz_xw_s += std::min(32 * d.fz_cpl_s, d.out_mul[i]) * (2 * d.out_l[i] + 1);
+    auto bytes = [&](int xw) {
+      int Y = 2 * kEdgeBatch * 16, B = 2 * kEdgeBatch * d.rm, S = 2 * kEdgeBatch, T = 2 * kMaxBlocks;
+      int X = (Y + B + S + T + 3) & ~3;
+      return (X + 2 * kEdgeBatch * xw + msz) * 4;
+    };
+    d.fz_smem_f = bytes(d.fz_xw_f);
+    d.fz_smem_s = bytes(d.fz_xw_s);
+  }
+  // lane-per-edge adjoint stream: channel tile cw (multiple of 4) chosen as large as fits
+  {
+    bool ok = true;
+    for (int i = 0; i < d.n_in; ++i) ok = ok && (d.in_mul[i] % 4 == 0);
+    for (int i = 0; i < d.n_out; ++i) ok = ok && (d.Kb[i] % 4 == 0);
+    d.adj_cw = 0;
+    if (ok) {
+      int acc = 0, rn3 = 0;
+      for (int i = 0; i < P; ++i) {
+        d.path[i].adj_goff = rn3;
+        rn3 += R * (2 * d.path[i].l3 + 1);
+        d.path[i].adj_acc = acc;
+        acc += 32 * ((2 * d.path[i].l2 + 1) + d.rm);
+      }
+      const int cmax = (d.max_c_in + 3) & ~3;
+      const int cands[6] = {cmax, 128, 64, 32, 16, 4};
+      for (int c : cands) {
+        if (c > cmax || c <= 0) continue;
+        int xw = 0;
+        for (int i = 0; i < d.n_in; ++i) xw += std::min(c, d.in_mul[i]) * (2 * d.in_l[i] + 1);
+        const int xs = xw | 1;
+        const int g = rn3 * c;
+        const int head = g + 32 * xs + 32 * 16 + 32 * d.rm + 32;
+        const int bytes = (((head + 3) & ~3) + acc) * 4;
+        if (bytes <= 227 * 1024) {
+          d.adj_cw = c;
+          d.adj_g = g;
+          d.adj_xs = xs;
+          d.adj_smem = bytes;
+          break;
+        }
+      }
+    }
+  }
+  if (size_t(std::max(std::max(sm, sm2) * 4, std::max(d.fz_smem_f, d.fz_smem_s))) > 227 * 1024) {
     delete p;
     return TPCONV_ERR_UNSUPPORTED;
   }
@@ -445,7 +502,7 @@ int tpc::ws_layout(const tpconv_plan& p, int op, int64_t N, int64_t E, WsLayout*
   L->state_bytes = size_t(Nc) * size_t(per_node) * 4;
   off = align256(off + L->state_bytes);
   L->off_theta = off;
-  L->theta_bytes = align256(p.theta_numel * 4) * 2;
+  L->theta_bytes = align256(p.theta_numel * 4 * 4);  // Theta^T (hi, lo) and gg_Theta^T (hi, lo)
   off = align256(off + L->theta_bytes);
   L->total = off;
   return TPCONV_OK;

@@ -94,6 +94,9 @@ struct DevPath {
   int32_t nmz;              // m_count(l1, l2, l3)
   int32_t sm_off;           // float offset of this path's warp scratch (first-order adjoint stream)
   int32_t sm_off2;          // same for the double-backward adjoint stream
+  int32_t smf_off;          // float offset of this path's coupling-matrix scratch in the fused streams
+  int32_t adj_goff;         // adjoint stream: this path's G tile at adj_goff * channel-tile floats
+  int32_t adj_acc;          // adjoint stream: float offset of this path's per-edge partials
 };
 
 struct DevPlan {
@@ -111,6 +114,12 @@ struct DevPlan {
   int rm;                           // radial registers per lane (4, 8 or 16) >= R
   int sm_floats;                    // dynamic smem floats of the first-order adjoint stream
   int sm_floats2;                   // dynamic smem floats of the double-backward adjoint stream
+  int fz_warps;                     // warps per CTA of the fused streams (paths run in passes)
+  int fz_cpl_f, fz_xw_f;            // forward: channels per lane, staged x floats per edge
+  int fz_cpl_s, fz_xw_s;            // sender stream: channels per lane, staged g floats per edge
+  int fz_smem_f, fz_smem_s;         // dynamic smem bytes of the fused forward / sender streams
+  int adj_cw;                       // adjoint stream channel tile (0: lane-per-edge stream unavailable)
+  int adj_g, adj_xs, adj_smem;      // its G tile floats, staged row stride (odd), smem bytes
   DevPath path[kMaxPaths];
 };
 

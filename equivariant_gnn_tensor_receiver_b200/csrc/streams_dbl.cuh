@@ -53,26 +53,6 @@ __device__ __forceinline__ void geom_dir(const DevPlan& pl, const float* v, cons
   }
 }
 
-// compact coupling matrix of one degree-L2 vector into Mrow
-template <int L1, int L2, int L3>
-__device__ __forceinline__ void coupling_row(const float* Y, float* Mrow) {
-  using TR = Tri<L1, L2, L3>;
-  sfor<TR::N1>([&](auto I1) {
-    sfor<TR::N3>([&](auto I3) {
-      constexpr int i1 = decltype(I1)::value, i3 = decltype(I3)::value;
-      if constexpr (TR::tab.m[i1][i3]) {
-        float s = 0.f;
-        sfor<TR::N2>([&](auto I2) {
-          constexpr int i2 = decltype(I2)::value;
-          if constexpr (TR::tab.cg[i1][i2][i3]) s = fmaf(TR::template cg<i1, i2, i3>(), Y[i2], s);
-        });
-        constexpr int mi = TR::tab.mi[i1][i3];
-        Mrow[mi] = s;
-      }
-    });
-  });
-}
-
 // per-batch preparation (lane = edge): M, Mdot, b, bdot into warp scratch
 template <int L1, int L2, int L3, int RM>
 __device__ __forceinline__ void prep_edge_dir(const DevPlan& pl, const float* v, const float* u, float* sM,

@@ -19,12 +19,20 @@
 #include <vector>
 
 #include "gemm_simt.cuh"
+#include "gemm_tc.h"
 #include "graph.cuh"
 #include "launchers.h"
 #include "plan.h"
 #include "workspace.h"
 
 using namespace tpc;
+
+namespace tpc {
+std::vector<TuInit>& tu_registry() {
+  static std::vector<TuInit> r;
+  return r;
+}
+}  // namespace tpc
 
 namespace {
 
@@ -42,8 +50,10 @@ int ensure_device() {
   if (g_ready[dev]) return TPCONV_OK;
   const float* t = cg_table_f32();
   if (!t) return TPCONV_ERR_INTERNAL;
-  if (upload_cg_fwd(t) || upload_cg_send(t) || upload_cg_radj(t) || upload_cg_dbl(t)) return TPCONV_ERR_CUDA;
-  if (radj_set_smem_limit(227 * 1024) || dbl_set_smem_limit(227 * 1024)) return TPCONV_ERR_CUDA;
+  for (const TuInit& tu : tu_registry()) {
+    if (tu.upload(t) != cudaSuccess) return TPCONV_ERR_CUDA;
+    if (tu.smem && tu.smem(227 * 1024) != cudaSuccess) return TPCONV_ERR_CUDA;
+  }
   g_ready[dev] = true;
   return TPCONV_OK;
 }
@@ -102,17 +112,48 @@ int check_ws(const tpconv_plan* plan, int op, int64_t N, int64_t E, void* ws, si
   return TPCONV_OK;
 }
 
-// out[r0 : r0+nc] = A . Theta (mode 0) or += (mode 1), per output block
-cudaError_t node_mix_forward(const DevPlan& d, int r0, int nc, const float* A, const float* theta, float* out,
-                             cudaStream_t st, int mode = 0) {
+// Theta^T of every output block (tensor-core B operand): hi (and lo for 3xTF32)
+// at the block's Theta offset inside the workspace's Theta region.
+cudaError_t prep_theta_T(const tpconv_plan* plan, const float* theta, float* hi, float* lo, cudaStream_t st) {
+  const DevPlan& d = plan->dp;
+  for (int i3 = 0; i3 < d.n_out; ++i3) {
+    const int p0 = first_path_of_out_block(d, i3);
+    if (p0 < 0) continue;
+    const int64_t off = d.path[p0].theta_off;
+    cudaError_t e = split_transpose(theta + off, d.Kb[i3], d.out_mul[i3], hi + off, lo ? lo + off : nullptr, st);
+    if (e) return e;
+  }
+  return cudaSuccess;
+}
+
+bool use_tc(const tpconv_plan* plan) {
+  return plan->opt.gemm == TPCONV_GEMM_FP32 || plan->opt.gemm == TPCONV_GEMM_TF32;
+}
+
+// out[r0 : r0+nc] = A . Theta (mode 0) or += (mode 1), per output block.  With
+// thT (Theta^T hi, lo) the tensor-core GEMM runs, else the FFMA GEMM.
+cudaError_t node_mix_forward(const tpconv_plan* plan, int r0, int nc, const float* A, const float* theta,
+                             const float* thT_hi, const float* thT_lo, float* out, cudaStream_t st, int mode = 0) {
+  const DevPlan& d = plan->dp;
   for (int i3 = 0; i3 < d.n_out; ++i3) {
     const int n3 = 2 * d.out_l[i3] + 1, cout = d.out_mul[i3];
     const int p0 = first_path_of_out_block(d, i3);
-    const float* th = theta + (p0 >= 0 ? d.path[p0].theta_off : 0);
-    MView a = mrow(F(A) + size_t(nc) * d.a_pref[i3], d.Kb[i3]);
-    MView b = mrow(F(th), cout);
+    const int64_t toff = p0 >= 0 ? d.path[p0].theta_off : 0;
+    const float* Ab = A + size_t(nc) * d.a_pref[i3];
+    const int Kb = d.Kb[i3];
+    const int64_t M = int64_t(nc) * n3;
+    if (thT_hi && Kb > 0 && gemm_tc_supported(Ab, Kb, thT_hi + toff, Kb, int(M), cout, Kb)) {
+      TcOut o{out + size_t(r0) * d.dim_out + d.out_off[i3], n3, d.dim_out, 1, n3};
+      const bool split = plan->opt.gemm == TPCONV_GEMM_FP32;
+      cudaError_t e = gemm_tc(Ab, Kb, thT_hi + toff, split ? thT_lo + toff : nullptr, Kb, int(M), cout, Kb, o,
+                              mode, split, st);
+      if (e) return e;
+      continue;
+    }
+    MView a = mrow(F(Ab), Kb);
+    MView b = mrow(F(theta + toff), cout);
     MView c = mview(out + size_t(r0) * d.dim_out + d.out_off[i3], n3, d.dim_out, 1, 1, n3, 0);
-    cudaError_t e = gemm_simt(int64_t(nc) * n3, cout, d.Kb[i3], a, b, c, mode, st);
+    cudaError_t e = gemm_simt(M, cout, Kb, a, b, c, mode, st);
     if (e) return e;
   }
   return cudaSuccess;
@@ -253,16 +294,27 @@ int tpconv_forward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t*
   const DevPlan& d = plan->dp;
   cudaStream_t s = S(stream);
   float* A = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_state);
+  float* thT = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_theta);
+  float* thT_hi = nullptr;
+  float* thT_lo = nullptr;
+  if (use_tc(plan)) {
+    PhaseScope ps(TPCONV_PHASE_OTHER, s);
+    thT_hi = thT;
+    thT_lo = thT + plan->theta_numel;
+    if (prep_theta_T(plan, theta, thT_hi, plan->opt.gemm == TPCONV_GEMM_FP32 ? thT_lo : nullptr, s))
+      return TPCONV_ERR_CUDA;
+    note(TPCONV_PHASE_OTHER, d.n_out);
+  }
   for (int64_t r0 = 0; r0 < N; r0 += L.chunk_nodes) {
     const int nc = int(std::min<int64_t>(L.chunk_nodes, N - r0));
     {
       PhaseScope ps(TPCONV_PHASE_FWD_EDGE, s);
-      if (launch_fwd_stream(d, int(r0), nc, rowptr, col, edge_vec, x, A, s)) return TPCONV_ERR_CUDA;
+      if (TPC_RM_CALL(d.rm, launch_fwd_rm, d, int(r0), nc, rowptr, col, edge_vec, x, A, s)) return TPCONV_ERR_CUDA;
       note(TPCONV_PHASE_FWD_EDGE, d.P);
     }
     {
       PhaseScope ps(TPCONV_PHASE_FWD_NODE, s);
-      if (node_mix_forward(d, int(r0), nc, A, theta, out, s)) return TPCONV_ERR_CUDA;
+      if (node_mix_forward(plan, int(r0), nc, A, theta, thT_hi, thT_lo, out, s)) return TPCONV_ERR_CUDA;
       note(TPCONV_PHASE_FWD_NODE, d.n_out);
     }
   }
@@ -299,8 +351,12 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
       }
       {
         PhaseScope ps(TPCONV_PHASE_BWD_EDGE_R, s);
-        if (launch_radj_stream(d, int(r0), nc, rowptr, col, edge_vec, x, S_, dvec, dY, db, s))
-          return TPCONV_ERR_CUDA;
+        cudaError_t e = d.adj_cw > 0
+                            ? TPC_RM_CALL(d.rm, launch_adj_rm, d, int(r0), nc, rowptr, col, edge_vec, x, S_, dvec, dY,
+                                          db, s)
+                            : TPC_RM_CALL(d.rm, launch_radj_rm, d, int(r0), nc, rowptr, col, edge_vec, x, S_, dvec,
+                                          dY, db, s);
+        if (e) return TPCONV_ERR_CUDA;
         note(TPCONV_PHASE_BWD_EDGE_R, 1);
       }
     }
@@ -310,7 +366,7 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
       const int nc = int(std::min<int64_t>(L.chunk_nodes, N - s0));
       {
         PhaseScope ps(TPCONV_PHASE_BWD_EDGE_S, s);
-        if (launch_send_stream(d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, g, S_, s)) return TPCONV_ERR_CUDA;
+        if (TPC_RM_CALL(d.rm, launch_send_rm, d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, g, S_, s)) return TPCONV_ERR_CUDA;
         note(TPCONV_PHASE_BWD_EDGE_S, d.P);
       }
       {
@@ -350,19 +406,32 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
   if (d_g) {
     float* A1 = W0;
     float* A0 = W0 + size_t(Nc) * plan->a_floats;
+    float* thT = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_theta);
+    float *t_hi = nullptr, *t_lo = nullptr, *gt_hi = nullptr, *gt_lo = nullptr;
+    if (use_tc(plan)) {
+      PhaseScope ps(TPCONV_PHASE_OTHER, s);
+      const bool split = plan->opt.gemm == TPCONV_GEMM_FP32;
+      t_hi = thT;
+      t_lo = thT + plan->theta_numel;
+      gt_hi = thT + 2 * plan->theta_numel;
+      gt_lo = thT + 3 * plan->theta_numel;
+      if (prep_theta_T(plan, theta, t_hi, split ? t_lo : nullptr, s)) return TPCONV_ERR_CUDA;
+      if (has_t && prep_theta_T(plan, gg_theta, gt_hi, split ? gt_lo : nullptr, s)) return TPCONV_ERR_CUDA;
+      note(TPCONV_PHASE_OTHER, d.n_out * (has_t ? 2 : 1));
+    }
     for (int64_t r0 = 0; r0 < N; r0 += Nc) {
       const int nc = int(std::min<int64_t>(Nc, N - r0));
       {
         PhaseScope ps(TPCONV_PHASE_DBL_EDGE_A, s);
-        if (launch_dbl_a_stream(d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, A1, A0, s))
+        if (TPC_RM_CALL(d.rm, launch_dbl_a_rm, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, A1, A0, s))
           return TPCONV_ERR_CUDA;
         note(TPCONV_PHASE_DBL_EDGE_A, d.P);
       }
       PhaseScope ps(TPCONV_PHASE_DBL_NODE_A, s);
-      if (node_mix_forward(d, int(r0), nc, A1, theta, d_g, s, 0)) return TPCONV_ERR_CUDA;
+      if (node_mix_forward(plan, int(r0), nc, A1, theta, t_hi, t_lo, d_g, s, 0)) return TPCONV_ERR_CUDA;
       note(TPCONV_PHASE_DBL_NODE_A, d.n_out);
       if (has_t) {
-        if (node_mix_forward(d, int(r0), nc, A0, gg_theta, d_g, s, 1)) return TPCONV_ERR_CUDA;
+        if (node_mix_forward(plan, int(r0), nc, A0, gg_theta, gt_hi, gt_lo, d_g, s, 1)) return TPCONV_ERR_CUDA;
         note(TPCONV_PHASE_DBL_NODE_A, d.n_out);
       }
     }
@@ -383,8 +452,8 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
         }
       }
       PhaseScope ps(TPCONV_PHASE_DBL_EDGE_R, s);
-      if (launch_dbl_r_stream(d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, G, has_t ? Gt : nullptr,
-                              d_vec, s))
+      if (TPC_RM_CALL(d.rm, launch_dbl_r_rm, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, G,
+                      has_t ? Gt : nullptr, d_vec, s))
         return TPCONV_ERR_CUDA;
       note(TPCONV_PHASE_DBL_EDGE_R, 1);
     }
@@ -397,7 +466,7 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
       const int nc = int(std::min<int64_t>(Nc, N - s0));
       {
         PhaseScope ps(TPCONV_PHASE_DBL_EDGE_S, s);
-        if (launch_dbl_s_stream(d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, gg_vec, g, B1, B0, s))
+        if (TPC_RM_CALL(d.rm, launch_dbl_s_rm, d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, gg_vec, g, B1, B0, s))
           return TPCONV_ERR_CUDA;
         note(TPCONV_PHASE_DBL_EDGE_S, d.P);
       }

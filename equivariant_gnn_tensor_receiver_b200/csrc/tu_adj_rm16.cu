@@ -1,0 +1,9 @@
+// Lane-per-edge receiver adjoint stream, radial width 16.
+#include "launch_adj.cuh"
+#include "launch_streams.cuh"
+
+namespace tpc {
+template cudaError_t launch_adj_rm<16>(const DevPlan&, int, int, const int*, const int*, const float*,
+                                       const float*, const float*, float*, float*, float*, cudaStream_t);
+}  // namespace tpc
+TPC_REGISTER_TU(adj_rm16, &tpc::adj_smem_rm<16>)

@@ -1,0 +1,8 @@
+// Fused forward receiver stream, radial width 8.
+#include "launch_fused.cuh"
+
+namespace tpc {
+template cudaError_t launch_fwd_rm<8>(const DevPlan&, int, int, const int*, const int*, const float*,
+                                       const float*, float*, cudaStream_t);
+}  // namespace tpc
+TPC_REGISTER_TU(fused_fwd_rm8, &tpc::fwd_fused_smem_rm<8>)

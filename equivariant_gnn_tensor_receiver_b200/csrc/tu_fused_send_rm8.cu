@@ -1,0 +1,8 @@
+// Fused backward sender stream, radial width 8.
+#include "launch_fused.cuh"
+
+namespace tpc {
+template cudaError_t launch_send_rm<8>(const DevPlan&, int, int, const int*, const int*, const int*,
+                                        const float*, const float*, float*, cudaStream_t);
+}  // namespace tpc
+TPC_REGISTER_TU(fused_send_rm8, &tpc::send_fused_smem_rm<8>)

@@ -14,6 +14,8 @@ from oracle import conv
 pytestmark = pytest.mark.gpu
 
 TOL_FP32 = 1e-5
+TOL_LOWP = 5e-3
+TOL = {"simt": TOL_FP32, "fp32": TOL_FP32, "tf32": TOL_LOWP}
 
 
 @pytest.fixture(scope="module")
@@ -135,15 +137,18 @@ def test_graph_transpose_exact(T):
     assert np.array_equal(s_rowptr, np.concatenate([[0], np.cumsum(np.bincount(col, minlength=N))]))
 
 
-def test_mace_full_size_sampled(T):
+@pytest.mark.parametrize("gemm", ["fp32", "tf32", "simt"])
+def test_mace_full_size_sampled(T, gemm):
     """The mace layer at full size (4096 atoms, ~214k edges), forward and the
     per-edge / per-sender adjoints checked on sampled receivers, edges and
-    senders, each of which the oracle computes exactly from its own edges."""
+    senders, each of which the oracle computes exactly from its own edges.
+    gemm selects the node-level Theta contraction: 3xTF32 or TF32 tensor cores
+    (tcgen05) or FFMA."""
     import torch
     c = W.CONFIGS["mace"]
     graph = W.graph_for("mace", 0)
     plan, prob, G, inp = make(T, c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], c["radial"],
-                              c["radial_params"], graph, seed=41)
+                              c["radial_params"], graph, seed=41, gemm=gemm)
     rowptr, col, vec, x, th, g = inp
     out, bw = run_fwd_bwd(T, plan, G, inp)
     N = len(rowptr) - 1
@@ -154,7 +159,7 @@ def test_mace_full_size_sampled(T):
     Y, b, JY, Jb = conv.geometry(prob, vec[em], order=1)
     ref = conv.forward_core(prob, len(rs), col[em].astype(np.int64), np.array([loc[r] for r in recv[em]]), x, Y,
                             b, th)
-    assert rel(out[rs], ref) < TOL_FP32
+    assert rel(out[rs], ref) < TOL[gemm], rel(out[rs], ref)
     # per-edge adjoints of the sampled receivers' edges (local quantities)
     gl = g[rs]
     _, _, dY, db = conv.backward_core(prob, len(rs), col[em].astype(np.int64),
@@ -199,3 +204,26 @@ def test_double_backward_parity(T, case):
             assert np.abs(got).max() == 0, k
         else:
             assert rel(got, ref[k]) < TOL_FP32, (k, rel(got, ref[k]))
+
+
+@pytest.mark.parametrize("gemm", ["fp32", "tf32"])
+@pytest.mark.parametrize("irr", ["16x0e+16x1o+16x2e", "24x0e+40x1o"])
+def test_tensor_core_mixing(T, gemm, irr):
+    """Forward through the tcgen05 Theta contraction: M = nodes x (2l+1) with a
+    ragged last 128-row tile, C_out below / between the 32..256 column tiles."""
+    import torch
+    graph = W.radius_graph(333, 15.0, 5.0, 8)
+    plan, prob, G, inp = make(T, irr, 2, irr, 8, "bessel", (5.0,), graph, seed=61, gemm=gemm)
+    rowptr, col, vec, x, th, g = inp
+    out = T.forward(plan, G, dev(x, torch.float32), dev(th, torch.float32))
+    torch.cuda.synchronize()
+    ref = conv.forward(prob, rowptr, col, vec, x, th)
+    assert rel(out.cpu().numpy(), ref) < TOL[gemm]
+    dbl = T.double_backward(plan, G, dev(x, torch.float32), dev(th, torch.float32), dev(g, torch.float32),
+                            dev(W.normal(x.shape, 62), torch.float32), dev(W.normal(vec.shape, 63), torch.float32),
+                            dev(W.normal(th.shape, 64) * 0.05, torch.float32), want=("d_g",))
+    torch.cuda.synchronize()
+    r32 = lambda a: a.astype(np.float32).astype(np.float64)
+    refd = conv.double_backward(prob, rowptr, col, vec, x, th, g, r32(W.normal(x.shape, 62)),
+                                r32(W.normal(vec.shape, 63)), r32(W.normal(th.shape, 64) * 0.05))
+    assert rel(dbl["d_g"].cpu().numpy(), refd["d_g"]) < TOL[gemm]
