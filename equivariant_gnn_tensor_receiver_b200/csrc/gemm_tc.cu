@@ -29,6 +29,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -153,13 +154,25 @@ struct TcSmem {
   static constexpr int kBytes = kStages * kStage + 1024 /*align*/ + 256 /*barriers*/;
 };
 
+// Accumulators in TMEM: the 3xTF32 mode spreads consecutive K steps over NACC
+// accumulators (summed in fp32 by the epilogue), so each one sees 1/NACC of
+// the accumulation steps; this bounds the error the accumulation itself adds.
+template <int BN, bool SPLIT>
+struct TcAcc {
+  static constexpr int kCols = BN < 32 ? 32 : BN;
+  static constexpr int N = SPLIT ? (512 / kCols > 8 ? 8 : 512 / kCols) : 1;
+  static constexpr uint32_t kAlloc = kCols * N;  // power of two, <= 512
+};
+
 template <int BN, bool SPLIT>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmBlo, int M, int N, int K, TcOut out, int accumulate) {
   using SM = TcSmem<BN>;
   constexpr int S = SM::kStages;
-  constexpr uint32_t kCols = BN < 32 ? 32 : BN;
+  constexpr uint32_t kCols = TcAcc<BN, SPLIT>::kCols;
+  constexpr int NACC = TcAcc<BN, SPLIT>::N;
+  constexpr uint32_t kAlloc = TcAcc<BN, SPLIT>::kAlloc;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(base + S * SM::kStage);
@@ -186,7 +199,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(kCols));
+                 "r"(kAlloc));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   asm volatile("tcgen05.fence::before_thread_sync;");
@@ -230,13 +243,14 @@ __global__ void __launch_bounds__(192, 1)
         asm volatile("tcgen05.fence::after_thread_sync;");
         const uint32_t a = smem_u32(sA(s)), al = smem_u32(sAlo(s)), b = smem_u32(sB(s)), bl = smem_u32(sBlo(s));
 #pragma unroll
+        const uint32_t td = tmem + uint32_t((kt % NACC) * kCols);
         for (int kk = 0; kk < kBK / 8; ++kk) {
           const uint32_t off = kk * 32;  // 8 TF32 = 32 bytes along K inside the swizzle atom
-          const uint32_t acc = (kt > 0 || kk > 0) ? 1u : 0u;
-          mma_tf32(tmem, sw128_desc(a + off), sw128_desc(b + off), idesc, acc);
+          const uint32_t acc = (kt >= NACC || kk > 0) ? 1u : 0u;
+          mma_tf32(td, sw128_desc(a + off), sw128_desc(b + off), idesc, acc);
           if (SPLIT) {
-            mma_tf32(tmem, sw128_desc(a + off), sw128_desc(bl + off), idesc, 1u);
-            mma_tf32(tmem, sw128_desc(al + off), sw128_desc(b + off), idesc, 1u);
+            mma_tf32(td, sw128_desc(a + off), sw128_desc(bl + off), idesc, 1u);
+            mma_tf32(td, sw128_desc(al + off), sw128_desc(b + off), idesc, 1u);
           }
         }
         mma_commit(&empty[s]);
@@ -279,17 +293,41 @@ __global__ void __launch_bounds__(192, 1)
       const int q = warp & 3;  // TMEM lane quadrant this warp may access
       const int row = m0 + q * 32 + lane;
       const int64_t rbase = (row / out.rdiv) * out.r_hi + (row % out.rdiv) * out.r_lo;
+      const int nacc = nk < NACC ? nk : NACC;  // accumulators that received a K step
 #pragma unroll 1
       for (int c = 0; c < BN; c += 16) {
         float v[16];
         tmem_ld16<BN>(tmem + (uint32_t(q * 32) << 16) + uint32_t(c), v);
-        if (row < M) {
+        for (int a = 1; a < nacc; ++a) {
+          float w[16];
+          tmem_ld16<BN>(tmem + (uint32_t(q * 32) << 16) + uint32_t(a * kCols + c), w);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int col = n0 + c + i;
-            if (col < N) {
-              float* dst = out.p + rbase + int64_t(col) * out.c_hi;
-              *dst = accumulate ? *dst + v[i] : v[i];
+          for (int i = 0; i < 16; ++i) v[i] += w[i];
+        }
+        if (row < M) {
+          float* dst0 = out.p + rbase + int64_t(n0 + c) * out.c_hi;
+          if (out.c_hi == 1 && n0 + c + 16 <= N && (reinterpret_cast<uintptr_t>(dst0) & 15) == 0) {
+            float4* d4 = reinterpret_cast<float4*>(dst0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              float4 t = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+              if (accumulate) {
+                const float4 o = d4[i];
+                t.x += o.x;
+                t.y += o.y;
+                t.z += o.z;
+                t.w += o.w;
+              }
+              d4[i] = t;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int col = n0 + c + i;
+              if (col < N) {
+                float* dst = out.p + rbase + int64_t(col) * out.c_hi;
+                *dst = accumulate ? *dst + v[i] : v[i];
+              }
             }
           }
         }
@@ -305,7 +343,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   if (warp == 1) {
     asm volatile("tcgen05.fence::after_thread_sync;");
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kAlloc));
   }
 }
 
@@ -428,6 +466,79 @@ __global__ void k_split_transpose(const float* __restrict__ th, int K, int N, fl
 cudaError_t split_transpose(const float* th, int K, int N, float* hi, float* lo, cudaStream_t st) {
   dim3 grid(unsigned((K + 31) / 32), unsigned((N + 31) / 32));
   k_split_transpose<<<grid, dim3(32, 8), 0, st>>>(th, K, N, hi, lo);
+  return cudaGetLastError();
+}
+
+// elementwise split: hi = rn_tf32(v), lo = rn_tf32(v - hi)  (lo may be null: hi = v)
+__global__ void k_split(const float* __restrict__ v, int64_t n, float* __restrict__ hi, float* __restrict__ lo) {
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const float a = v[i];
+    if (lo) {
+      const float h = rn_tf32(a);
+      hi[i] = h;
+      lo[i] = rn_tf32(a - h);
+    } else {
+      hi[i] = a;
+    }
+  }
+}
+
+cudaError_t split_elementwise(const float* v, int64_t n, float* hi, float* lo, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  const int blocks = int(std::min<int64_t>((n + 255) / 256, 148 * 8));
+  k_split<<<blocks, 256, 0, st>>>(v, n, hi, lo);
+  return cudaGetLastError();
+}
+
+// Theta of the paths of input block i1 as [c_in][K_x] with column kxoff(p) + k*c_out + w
+// (dx = B . Theta operand); optional TF32 split.
+__global__ void k_theta_x(const float* __restrict__ th, int64_t theta_off, int R, int c_in, int c_out, int kxoff,
+                          int Kx, float* __restrict__ hi, float* __restrict__ lo) {
+  const int64_t n = int64_t(R) * c_in * c_out;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const int w = int(i % c_out);
+    const int64_t t = i / c_out;
+    const int u = int(t % c_in), k = int(t / c_in);
+    const float a = th[theta_off + i];  // Theta[p][k][u][w]
+    const int64_t o = int64_t(u) * Kx + kxoff + int64_t(k) * c_out + w;
+    if (lo) {
+      const float h = rn_tf32(a);
+      hi[o] = h;
+      lo[o] = rn_tf32(a - h);
+    } else {
+      hi[o] = a;
+    }
+  }
+}
+
+cudaError_t theta_x_pack(const float* th, int64_t theta_off, int R, int c_in, int c_out, int kxoff, int Kx, float* hi,
+                         float* lo, cudaStream_t st) {
+  const int64_t n = int64_t(R) * c_in * c_out;
+  if (n <= 0) return cudaSuccess;
+  const int blocks = int(std::min<int64_t>((n + 255) / 256, 148 * 8));
+  k_theta_x<<<blocks, 256, 0, st>>>(th, theta_off, R, c_in, c_out, kxoff, Kx, hi, lo);
+  return cudaGetLastError();
+}
+
+// g block of output block (offset, mul, 2l+1) of nodes r0 : r0+nc as [(node, m)][w]
+__global__ void k_pack_rows(const float* __restrict__ g, int dim, int off, int mul, int n3, int64_t r0, int nc,
+                            float* __restrict__ out) {
+  const int64_t total = int64_t(nc) * n3 * mul;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
+    const int w = int(i % mul);
+    const int64_t rm = i / mul;
+    const int m = int(rm % n3);
+    const int64_t r = rm / n3;
+    out[i] = g[(r0 + r) * dim + off + int64_t(w) * n3 + m];
+  }
+}
+
+cudaError_t pack_rows(const float* g, int dim, int off, int mul, int n3, int64_t r0, int nc, float* out,
+                      cudaStream_t st) {
+  const int64_t total = int64_t(nc) * n3 * mul;
+  if (total <= 0) return cudaSuccess;
+  const int blocks = int(std::min<int64_t>((total + 255) / 256, 148 * 16));
+  k_pack_rows<<<blocks, 256, 0, st>>>(g, dim, off, mul, n3, r0, nc, out);
   return cudaGetLastError();
 }
 

@@ -22,6 +22,17 @@ cudaError_t gemm_tc(const float* A, int64_t lda, const float* B, const float* Bl
 // Theta block [K][N] -> hi = its transpose [N][K] (rounded to TF32 when lo != null), lo = remainder.
 cudaError_t split_transpose(const float* th, int K, int N, float* hi, float* lo, cudaStream_t st);
 
+// hi = rn_tf32(v), lo = rn_tf32(v - hi) elementwise (lo null: plain copy)
+cudaError_t split_elementwise(const float* v, int64_t n, float* hi, float* lo, cudaStream_t st);
+
+// Theta[p] ([R][c_in][c_out]) into columns kxoff + k*c_out + w of a [c_in][Kx] matrix (split when lo != null)
+cudaError_t theta_x_pack(const float* th, int64_t theta_off, int R, int c_in, int c_out, int kxoff, int Kx, float* hi,
+                         float* lo, cudaStream_t st);
+
+// rows (node, m) x columns w of one feature block of nodes r0 : r0+nc -> dense [nc*n3][mul]
+cudaError_t pack_rows(const float* g, int dim, int off, int mul, int n3, int64_t r0, int nc, float* out,
+                      cudaStream_t st);
+
 // First error recorded by a bounded wait inside a tensor-core GEMM (0 = none); clears it. Synchronises st.
 cudaError_t gemm_tc_read_error(int* code, cudaStream_t st);
 

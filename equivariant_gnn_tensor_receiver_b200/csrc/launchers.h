@@ -37,6 +37,11 @@ cudaError_t launch_radj_rm(const DevPlan& d, int r0, int nc, const int* rowptr, 
 template <int RM>
 cudaError_t launch_adj_rm(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,
                           const float* x, const float* G, float* dvec, float* dY, float* db, cudaStream_t st);
+// double backward, lane-per-edge adjoint stream (requires plan.dadj_cw > 0)
+template <int RM>
+cudaError_t launch_dadj_rm(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,
+                           const float* ggv, const float* x, const float* ggx, const float* G, const float* Gt,
+                           float* dvec, cudaStream_t st);
 // double backward: [A1 | A0] of receivers r0 : r0+nc
 template <int RM>
 cudaError_t launch_dbl_a_rm(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,

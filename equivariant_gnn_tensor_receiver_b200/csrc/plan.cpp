@@ -384,6 +384,28 @@ int tpconv_plan_create(tpconv_plan** out, const char* irreps_in, int l_sh_max,
       }
       const int cmax = (d.max_c_in + 3) & ~3;
       const int cands[6] = {cmax, 128, 64, 32, 16, 4};
+      int dacc = 0;
+      for (int i = 0; i < P; ++i) {
+        d.path[i].dadj_acc = dacc;
+        dacc += 32 * (2 * (2 * d.path[i].l2 + 1) + 2 * d.rm);
+      }
+      d.dadj_cw = 0;
+      for (int c : cands) {
+        if (c > cmax || c <= 0) continue;
+        int xw = 0;
+        for (int i = 0; i < d.n_in; ++i) xw += std::min(c, d.in_mul[i]) * (2 * d.in_l[i] + 1);
+        const int xs = xw | 1;
+        const int g = rn3 * c;
+        const int head = 2 * g + 2 * 32 * xs + 2 * 32 * 16 + 2 * 32 * d.rm + 32;
+        const int bytes = (((head + 3) & ~3) + dacc) * 4;
+        if (bytes <= 227 * 1024) {
+          d.dadj_cw = c;
+          d.dadj_g = g;
+          d.dadj_xs = xs;
+          d.dadj_smem = bytes;
+          break;
+        }
+      }
       for (int c : cands) {
         if (c > cmax || c <= 0) continue;
         int xw = 0;
@@ -502,8 +524,11 @@ int tpc::ws_layout(const tpconv_plan& p, int op, int64_t N, int64_t E, WsLayout*
   L->state_bytes = size_t(Nc) * size_t(per_node) * 4;
   off = align256(off + L->state_bytes);
   L->off_theta = off;
-  L->theta_bytes = align256(p.theta_numel * 4 * 4);  // Theta^T (hi, lo) and gg_Theta^T (hi, lo)
+  L->theta_bytes = align256(((p.theta_numel + 63) & ~size_t(63)) * 4 * 12);  // 2 Thetas x {T, N, X} x {hi, lo}
   off = align256(off + L->theta_bytes);
+  L->off_pack = off;
+  L->pack_bytes = align256(size_t(Nc) * size_t(p.dp.dim_out) * 4);
+  off = align256(off + L->pack_bytes);
   L->total = off;
   return TPCONV_OK;
 }

@@ -97,6 +97,7 @@ struct DevPath {
   int32_t smf_off;          // float offset of this path's coupling-matrix scratch in the fused streams
   int32_t adj_goff;         // adjoint stream: this path's G tile at adj_goff * channel-tile floats
   int32_t adj_acc;          // adjoint stream: float offset of this path's per-edge partials
+  int32_t dadj_acc;         // double-backward adjoint stream: same
 };
 
 struct DevPlan {
@@ -120,6 +121,7 @@ struct DevPlan {
   int fz_smem_f, fz_smem_s;         // dynamic smem bytes of the fused forward / sender streams
   int adj_cw;                       // adjoint stream channel tile (0: lane-per-edge stream unavailable)
   int adj_g, adj_xs, adj_smem;      // its G tile floats, staged row stride (odd), smem bytes
+  int dadj_cw, dadj_g, dadj_xs, dadj_smem;  // the same for the double-backward adjoint stream
   DevPath path[kMaxPaths];
 };
 

@@ -23,6 +23,11 @@ __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
                "l"(src)
                : "memory");
 }
+__device__ __forceinline__ void cp_async16_ca(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
@@ -82,16 +87,31 @@ __device__ __forceinline__ void fz_stage(const DevPlan& pl, const FzLay& L, floa
     reinterpret_cast<int*>(sm + L.S)[buf * kEdgeBatch + j] = nbr[jb + j];
   }
   float* X = sm + L.X + buf * kEdgeBatch * L.xw;
+  // 16-byte copies when every staged segment and row pitch is 16-byte aligned
+  bool vec4 = (L.xw & 3) == 0 && (src_dim & 3) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+  for (int i = 0; i < nblk && vec4; ++i) {
+    const int n = 2 * lval[i] + 1;
+    vec4 = ((blk_off[i] + c0 * n) & 3) == 0 && (sT[i] & 3) == 0 && ((sT[kMaxBlocks + i] * n) & 3) == 0;
+  }
   for (int i = 0; i < nblk; ++i) {
     const int w = sT[kMaxBlocks + i];
     if (w <= 0) continue;
     const int n = 2 * lval[i] + 1;
     const int len = w * n;
     const int so = blk_off[i] + c0 * n, dof = sT[i];
-    for (int idx = threadIdx.x; idx < nb * len; idx += blockDim.x) {
-      const int j = idx / len, o = idx - j * len;
-      const int s = nbr[jb + j];
-      cp_async4(X + j * L.xw + dof + o, src + size_t(s) * src_dim + so + o);
+    if (vec4) {
+      const int len4 = len >> 2;
+      for (int j = 0; j < nb; ++j) {
+        const float* row = src + size_t(nbr[jb + j]) * src_dim + so;
+        for (int o = threadIdx.x; o < len4; o += blockDim.x)
+          cp_async16_ca(X + j * L.xw + dof + 4 * o, row + 4 * o);
+      }
+    } else {
+      for (int idx = threadIdx.x; idx < nb * len; idx += blockDim.x) {
+        const int j = idx / len, o = idx - j * len;
+        const int s = nbr[jb + j];
+        cp_async4(X + j * L.xw + dof + o, src + size_t(s) * src_dim + so + o);
+      }
     }
   }
   cp_async_commit();

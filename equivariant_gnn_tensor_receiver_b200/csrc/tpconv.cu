@@ -159,37 +159,122 @@ cudaError_t node_mix_forward(const tpconv_plan* plan, int r0, int nc, const floa
   return cudaSuccess;
 }
 
-// G[r0 : r0+nc] = g . Theta^T  (per output block)
-cudaError_t node_mix_adjoint(const DevPlan& d, int r0, int nc, const float* g, const float* theta, float* G,
-                             cudaStream_t st) {
-  for (int i3 = 0; i3 < d.n_out; ++i3) {
-    if (d.Kb[i3] == 0) continue;
-    const int n3 = 2 * d.out_l[i3] + 1, cout = d.out_mul[i3];
-    const int p0 = first_path_of_out_block(d, i3);
-    MView a = mview(F(g) + size_t(r0) * d.dim_out + d.out_off[i3], n3, d.dim_out, 1, 1, n3, 0);
-    MView b = mview(F(theta) + d.path[p0].theta_off, 1, 1, 0, 1, cout, 0);
-    MView c = mrow(G + size_t(nc) * d.a_pref[i3], d.Kb[i3]);
-    cudaError_t e = gemm_simt(int64_t(nc) * n3, d.Kb[i3], cout, a, b, c, 0, st);
-    if (e) return e;
+// Theta operands of the tensor-core contractions for one Theta (slot 0: Theta,
+// slot 1: gg_Theta), carved from the workspace's Theta region:
+//   T  = per output block Theta_blk^T [C_out][K_b]   (out / d_g = A . Theta)
+//   N  = Theta itself, split elementwise              (G = g . Theta^T)
+//   X  = per input block [C_in][K_x]                  (dx = B . Theta)
+// hi / lo are the 3xTF32 halves; lo is null in TF32 mode.
+struct TcTheta {
+  const float *T_hi = nullptr, *T_lo = nullptr, *N_hi = nullptr, *N_lo = nullptr, *X_hi = nullptr, *X_lo = nullptr;
+};
+
+int64_t x_block_off(const DevPlan& d, int i1) {
+  int64_t o = 0;
+  for (int i = 0; i < i1; ++i) o += int64_t(d.in_mul[i]) * d.Kx[i];
+  return o;
+}
+
+cudaError_t prep_tc_theta(const tpconv_plan* plan, const float* theta, float* region, int slot, bool needT,
+                          bool needN, bool needX, TcTheta* o, cudaStream_t st) {
+  const DevPlan& d = plan->dp;
+  const size_t tn = (plan->theta_numel + 63) & ~size_t(63);
+  const bool split = plan->opt.gemm == TPCONV_GEMM_FP32;
+  float* b = region + size_t(slot) * 6 * tn;
+  cudaError_t e;
+  if (needT) {
+    if ((e = prep_theta_T(plan, theta, b, split ? b + tn : nullptr, st))) return e;
+    o->T_hi = b;
+    o->T_lo = split ? b + tn : nullptr;
+  }
+  if (needN) {
+    if ((e = split_elementwise(theta, int64_t(plan->theta_numel), b + 2 * tn, split ? b + 3 * tn : nullptr, st)))
+      return e;
+    o->N_hi = b + 2 * tn;
+    o->N_lo = split ? b + 3 * tn : nullptr;
+  }
+  if (needX) {
+    for (int p = 0; p < d.P; ++p) {
+      const DevPath& q = d.path[p];
+      const int64_t xo = x_block_off(d, q.i1);
+      if ((e = theta_x_pack(theta, q.theta_off, d.R, q.c_in, q.c_out, q.kxoff, d.Kx[q.i1], b + 4 * tn + xo,
+                            split ? b + 5 * tn + xo : nullptr, st)))
+        return e;
+    }
+    o->X_hi = b + 4 * tn;
+    o->X_lo = split ? b + 5 * tn : nullptr;
   }
   return cudaSuccess;
 }
 
-// dx[s0 : s0+nc] += B . Theta  and  dtheta += x^T B   (per path)
-cudaError_t node_mix_sender(const DevPlan& d, int s0, int nc, const float* B, const float* x, const float* theta,
-                            float* dx, float* dtheta, cudaStream_t st) {
-  for (int p = 0; p < d.P; ++p) {
-    const DevPath& q = d.path[p];
-    const int n1 = 2 * q.l1 + 1;
-    const int Kx = d.Kx[q.i1];
-    MView bp = mrow(F(B) + size_t(nc) * d.b_pref[q.i1] + q.kxoff, Kx);
+// G[r0 : r0+nc] = g . Theta^T  (per output block); gpack: nc * dim_out floats of scratch
+cudaError_t node_mix_adjoint(const tpconv_plan* plan, int r0, int nc, const float* g, const float* theta,
+                             const TcTheta* tc, float* gpack, float* G, cudaStream_t st) {
+  const DevPlan& d = plan->dp;
+  for (int i3 = 0; i3 < d.n_out; ++i3) {
+    if (d.Kb[i3] == 0) continue;
+    const int n3 = 2 * d.out_l[i3] + 1, cout = d.out_mul[i3];
+    const int p0 = first_path_of_out_block(d, i3);
+    const int64_t toff = d.path[p0].theta_off;
+    float* Gb = G + size_t(nc) * d.a_pref[i3];
+    const int64_t M = int64_t(nc) * n3;
     cudaError_t e;
-    if (dx) {
-      MView th = mview(F(theta) + q.theta_off, q.c_out, int64_t(q.c_in) * q.c_out, 1, 1, q.c_out, 0);
-      MView c = mview(dx + size_t(s0) * d.dim_in + q.in_off, n1, d.dim_in, 1, 1, n1, 0);
-      if ((e = gemm_simt(int64_t(nc) * n1, q.c_in, int64_t(d.R) * q.c_out, bp, th, c, 1, st))) return e;
+    if (tc && tc->N_hi && gemm_tc_supported(gpack, cout, tc->N_hi + toff, cout, int(M), d.Kb[i3], cout) &&
+        (d.Kb[i3] & 3) == 0) {
+      if ((e = pack_rows(g, d.dim_out, d.out_off[i3], cout, n3, r0, nc, gpack, st))) return e;
+      TcOut o{Gb, 1, d.Kb[i3], 0, 1};
+      const bool split = tc->N_lo != nullptr;
+      if ((e = gemm_tc(gpack, cout, tc->N_hi + toff, split ? tc->N_lo + toff : nullptr, cout, int(M), d.Kb[i3], cout,
+                       o, 0, split, st)))
+        return e;
+      continue;
     }
-    if (dtheta) {
+    MView a = mview(F(g) + size_t(r0) * d.dim_out + d.out_off[i3], n3, d.dim_out, 1, 1, n3, 0);
+    MView b = mview(F(theta) + toff, 1, 1, 0, 1, cout, 0);
+    MView c = mrow(Gb, d.Kb[i3]);
+    if ((e = gemm_simt(M, d.Kb[i3], cout, a, b, c, 0, st))) return e;
+  }
+  return cudaSuccess;
+}
+
+// dx[s0 : s0+nc] += B . Theta (per input block) and dtheta += x^T B (per path)
+cudaError_t node_mix_sender(const tpconv_plan* plan, int s0, int nc, const float* B, const float* x,
+                            const float* theta, const TcTheta* tc, float* dx, float* dtheta, cudaStream_t st) {
+  const DevPlan& d = plan->dp;
+  cudaError_t e;
+  if (dx) {
+    for (int i1 = 0; i1 < d.n_in; ++i1) {
+      const int Kx = d.Kx[i1];
+      if (Kx == 0) continue;
+      const int n1 = 2 * d.in_l[i1] + 1, cin = d.in_mul[i1];
+      const float* Bb = B + size_t(nc) * d.b_pref[i1];
+      const int64_t M = int64_t(nc) * n1;
+      if (tc && tc->X_hi) {
+        const int64_t xo = x_block_off(d, i1);
+        if (gemm_tc_supported(Bb, Kx, tc->X_hi + xo, Kx, int(M), cin, Kx)) {
+          TcOut o{dx + size_t(s0) * d.dim_in + d.in_off[i1], n1, d.dim_in, 1, n1};
+          const bool split = tc->X_lo != nullptr;
+          if ((e = gemm_tc(Bb, Kx, tc->X_hi + xo, split ? tc->X_lo + xo : nullptr, Kx, int(M), cin, Kx, o, 1, split,
+                           st)))
+            return e;
+          continue;
+        }
+      }
+      for (int p = 0; p < d.P; ++p) {
+        const DevPath& q = d.path[p];
+        if (q.i1 != i1) continue;
+        MView bp = mrow(F(B) + size_t(nc) * d.b_pref[q.i1] + q.kxoff, Kx);
+        MView th = mview(F(theta) + q.theta_off, q.c_out, int64_t(q.c_in) * q.c_out, 1, 1, q.c_out, 0);
+        MView c = mview(dx + size_t(s0) * d.dim_in + q.in_off, n1, d.dim_in, 1, 1, n1, 0);
+        if ((e = gemm_simt(M, q.c_in, int64_t(d.R) * q.c_out, bp, th, c, 1, st))) return e;
+      }
+    }
+  }
+  if (dtheta) {
+    for (int p = 0; p < d.P; ++p) {
+      const DevPath& q = d.path[p];
+      const int n1 = 2 * q.l1 + 1;
+      MView bp = mrow(F(B) + size_t(nc) * d.b_pref[q.i1] + q.kxoff, d.Kx[q.i1]);
       MView xa = mview(F(x) + size_t(s0) * d.dim_in + q.in_off, 1, n1, 0, n1, d.dim_in, 1);
       MView c = mview(dtheta + q.theta_off, 1, q.c_out, 0, q.c_out, int64_t(q.c_in) * q.c_out, 1);
       if ((e = gemm_simt(q.c_in, int64_t(d.R) * q.c_out, int64_t(nc) * n1, xa, bp, c, 2, st))) return e;
@@ -294,15 +379,15 @@ int tpconv_forward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t*
   const DevPlan& d = plan->dp;
   cudaStream_t s = S(stream);
   float* A = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_state);
-  float* thT = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_theta);
-  float* thT_hi = nullptr;
-  float* thT_lo = nullptr;
+  float* treg = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_theta);
+  const float* thT_hi = nullptr;
+  const float* thT_lo = nullptr;
   if (use_tc(plan)) {
     PhaseScope ps(TPCONV_PHASE_OTHER, s);
-    thT_hi = thT;
-    thT_lo = thT + plan->theta_numel;
-    if (prep_theta_T(plan, theta, thT_hi, plan->opt.gemm == TPCONV_GEMM_FP32 ? thT_lo : nullptr, s))
-      return TPCONV_ERR_CUDA;
+    TcTheta tc;
+    if (prep_tc_theta(plan, theta, treg, 0, true, false, false, &tc, s)) return TPCONV_ERR_CUDA;
+    thT_hi = tc.T_hi;
+    thT_lo = tc.T_lo;
     note(TPCONV_PHASE_OTHER, d.n_out);
   }
   for (int64_t r0 = 0; r0 < N; r0 += L.chunk_nodes) {
@@ -341,13 +426,23 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
   if (dx && N > 0 && cudaMemsetAsync(dx, 0, size_t(N) * d.dim_in * 4, s)) return TPCONV_ERR_CUDA;
   if (N == 0) return finish(cudaSuccess);
   float* S_ = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_state);
+  float* treg = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_theta);
+  float* gpack = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_pack);
+  TcTheta tc;
+  const TcTheta* tcp = nullptr;
+  if (use_tc(plan)) {
+    PhaseScope ps(TPCONV_PHASE_OTHER, s);
+    if (prep_tc_theta(plan, theta, treg, 0, false, want_edge && E > 0, dx != nullptr, &tc, s)) return TPCONV_ERR_CUDA;
+    note(TPCONV_PHASE_OTHER, 1 + d.P);
+    tcp = &tc;
+  }
   if (want_edge && E > 0) {
     for (int64_t r0 = 0; r0 < N; r0 += L.chunk_nodes) {
       const int nc = int(std::min<int64_t>(L.chunk_nodes, N - r0));
       {
         PhaseScope ps(TPCONV_PHASE_BWD_NODE_G, s);
-        if (node_mix_adjoint(d, int(r0), nc, g, theta, S_, s)) return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_BWD_NODE_G, d.n_out);
+        if (node_mix_adjoint(plan, int(r0), nc, g, theta, tcp, gpack, S_, s)) return TPCONV_ERR_CUDA;
+        note(TPCONV_PHASE_BWD_NODE_G, 2 * d.n_out);
       }
       {
         PhaseScope ps(TPCONV_PHASE_BWD_EDGE_R, s);
@@ -371,8 +466,8 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
       }
       {
         PhaseScope ps(TPCONV_PHASE_BWD_NODE_X, s);
-        if (node_mix_sender(d, int(s0), nc, S_, x, theta, dx, dtheta, s)) return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_BWD_NODE_X, int64_t(d.P) * ((dx ? 1 : 0) + (dtheta ? 1 : 0)));
+        if (node_mix_sender(plan, int(s0), nc, S_, x, theta, tcp, dx, dtheta, s)) return TPCONV_ERR_CUDA;
+        note(TPCONV_PHASE_BWD_NODE_X, int64_t(dx ? d.n_in : 0) + int64_t(dtheta ? d.P : 0));
       }
     }
   }
@@ -402,23 +497,29 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
   if (N == 0) return finish(cudaSuccess);
   float* W0 = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_state);
   const int64_t Nc = L.chunk_nodes;
+  float* treg = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_theta);
+  float* gpack = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_pack);
+  TcTheta tc0, tc1;
+  const TcTheta* tc0p = nullptr;
+  const TcTheta* tc1p = nullptr;
+  if (use_tc(plan)) {
+    PhaseScope ps(TPCONV_PHASE_OTHER, s);
+    const bool wantR = d_vec && E > 0;
+    if (prep_tc_theta(plan, theta, treg, 0, d_g != nullptr, wantR, d_x != nullptr, &tc0, s)) return TPCONV_ERR_CUDA;
+    tc0p = &tc0;
+    if (has_t) {
+      if (prep_tc_theta(plan, gg_theta, treg, 1, d_g != nullptr, wantR, d_x != nullptr, &tc1, s))
+        return TPCONV_ERR_CUDA;
+      tc1p = &tc1;
+    }
+    note(TPCONV_PHASE_OTHER, (has_t ? 2 : 1) * (d.n_out + 1 + d.P));
+  }
   // d_g = A1 . Theta + A0 . gg_theta
   if (d_g) {
     float* A1 = W0;
     float* A0 = W0 + size_t(Nc) * plan->a_floats;
-    float* thT = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_theta);
-    float *t_hi = nullptr, *t_lo = nullptr, *gt_hi = nullptr, *gt_lo = nullptr;
-    if (use_tc(plan)) {
-      PhaseScope ps(TPCONV_PHASE_OTHER, s);
-      const bool split = plan->opt.gemm == TPCONV_GEMM_FP32;
-      t_hi = thT;
-      t_lo = thT + plan->theta_numel;
-      gt_hi = thT + 2 * plan->theta_numel;
-      gt_lo = thT + 3 * plan->theta_numel;
-      if (prep_theta_T(plan, theta, t_hi, split ? t_lo : nullptr, s)) return TPCONV_ERR_CUDA;
-      if (has_t && prep_theta_T(plan, gg_theta, gt_hi, split ? gt_lo : nullptr, s)) return TPCONV_ERR_CUDA;
-      note(TPCONV_PHASE_OTHER, d.n_out * (has_t ? 2 : 1));
-    }
+    const float *t_hi = tc0p ? tc0.T_hi : nullptr, *t_lo = tc0p ? tc0.T_lo : nullptr;
+    const float *gt_hi = tc1p ? tc1.T_hi : nullptr, *gt_lo = tc1p ? tc1.T_lo : nullptr;
     for (int64_t r0 = 0; r0 < N; r0 += Nc) {
       const int nc = int(std::min<int64_t>(Nc, N - r0));
       {
@@ -444,17 +545,20 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
       const int nc = int(std::min<int64_t>(Nc, N - r0));
       {
         PhaseScope ps(TPCONV_PHASE_OTHER, s);
-        if (node_mix_adjoint(d, int(r0), nc, g, theta, G, s)) return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_OTHER, d.n_out);
+        if (node_mix_adjoint(plan, int(r0), nc, g, theta, tc0p, gpack, G, s)) return TPCONV_ERR_CUDA;
+        note(TPCONV_PHASE_OTHER, 2 * d.n_out);
         if (has_t) {
-          if (node_mix_adjoint(d, int(r0), nc, g, gg_theta, Gt, s)) return TPCONV_ERR_CUDA;
-          note(TPCONV_PHASE_OTHER, d.n_out);
+          if (node_mix_adjoint(plan, int(r0), nc, g, gg_theta, tc1p, gpack, Gt, s)) return TPCONV_ERR_CUDA;
+          note(TPCONV_PHASE_OTHER, 2 * d.n_out);
         }
       }
       PhaseScope ps(TPCONV_PHASE_DBL_EDGE_R, s);
-      if (TPC_RM_CALL(d.rm, launch_dbl_r_rm, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, G,
-                      has_t ? Gt : nullptr, d_vec, s))
-        return TPCONV_ERR_CUDA;
+      cudaError_t e = d.dadj_cw > 0
+                          ? TPC_RM_CALL(d.rm, launch_dadj_rm, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x,
+                                        gg_x, G, has_t ? Gt : nullptr, d_vec, s)
+                          : TPC_RM_CALL(d.rm, launch_dbl_r_rm, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x,
+                                        gg_x, G, has_t ? Gt : nullptr, d_vec, s);
+      if (e) return TPCONV_ERR_CUDA;
       note(TPCONV_PHASE_DBL_EDGE_R, 1);
     }
   }
@@ -473,12 +577,13 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
       PhaseScope ps(TPCONV_PHASE_DBL_NODE_X, s);
       float* dx1 = has_v ? d_x : nullptr;
       float* dt1 = has_v ? d_theta : nullptr;
-      if ((dx1 || dt1) && node_mix_sender(d, int(s0), nc, B1, x, theta, dx1, dt1, s)) return TPCONV_ERR_CUDA;
-      note(TPCONV_PHASE_DBL_NODE_X, int64_t(d.P) * ((dx1 ? 1 : 0) + (dt1 ? 1 : 0)));
+      if ((dx1 || dt1) && node_mix_sender(plan, int(s0), nc, B1, x, theta, tc0p, dx1, dt1, s)) return TPCONV_ERR_CUDA;
+      note(TPCONV_PHASE_DBL_NODE_X, int64_t(dx1 ? d.n_in : 0) + int64_t(dt1 ? d.P : 0));
       float* dx0 = has_t ? d_x : nullptr;
       float* dt0 = has_x1 ? d_theta : nullptr;
-      if ((dx0 || dt0) && node_mix_sender(d, int(s0), nc, B0, gg_x, gg_theta, dx0, dt0, s)) return TPCONV_ERR_CUDA;
-      note(TPCONV_PHASE_DBL_NODE_X, int64_t(d.P) * ((dx0 ? 1 : 0) + (dt0 ? 1 : 0)));
+      if ((dx0 || dt0) && node_mix_sender(plan, int(s0), nc, B0, gg_x, gg_theta, tc1p, dx0, dt0, s))
+        return TPCONV_ERR_CUDA;
+      note(TPCONV_PHASE_DBL_NODE_X, int64_t(dx0 ? d.n_in : 0) + int64_t(dt0 ? d.P : 0));
     }
   }
   return finish(cudaSuccess);

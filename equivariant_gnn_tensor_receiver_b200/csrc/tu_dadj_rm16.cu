@@ -1,0 +1,10 @@
+// Lane-per-edge double-backward adjoint stream, radial width 16.
+#include "launch_dadj.cuh"
+#include "launch_streams.cuh"
+
+namespace tpc {
+template cudaError_t launch_dadj_rm<16>(const DevPlan&, int, int, const int*, const int*, const float*,
+                                        const float*, const float*, const float*, const float*, const float*,
+                                        float*, cudaStream_t);
+}  // namespace tpc
+TPC_REGISTER_TU(dadj_rm16, &tpc::dadj_smem_rm<16>)

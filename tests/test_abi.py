@@ -83,5 +83,8 @@ def test_workspace_independent_of_edges_and_capped(T):
     assert len(sizes) == 1
     cap = 64 << 20
     capped = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], workspace_cap=cap)
+    theta_ops = 12 * 4 * capped.theta_numel  # tensor-core Theta operands: independent of N and E
     for op in (0, 1, 2):
-        assert T.tpconv_workspace_size(capped, op, 1_222_309, 64_000_000) < cap + (16 << 20)
+        big = T.tpconv_workspace_size(capped, op, 1_222_309, 64_000_000)
+        assert big == T.tpconv_workspace_size(capped, op, 500_000, 1_000)
+        assert big <= cap + theta_ops + (4 << 20)
