@@ -276,12 +276,19 @@ __device__ __forceinline__ void radial_basis(const DevPlan& pl, const T& r, T* b
       return;
     }
     T th = r * pl.rc0;                            // pi r / r_c
-    T fc = (dcos(th) + 1.f) * 0.5f;               // cosine cutoff
+    T c1 = dcos(th), s1 = dsin(th);
+    T fc = (c1 + 1.f) * 0.5f;                     // cosine cutoff (same angle)
     T pre = drecip(r) * fc * pl.rc1;              // sqrt(2/r_c) fc / r
+    // sin((k+1) th) = 2 cos(th) sin(k th) - sin((k-1) th): one sin/cos pair per edge
+    T c2 = c1 * 2.f;
+    T sp = T(0.f), sk = s1;
 #pragma unroll
     for (int k = 0; k < RM; ++k) {
-      if (k < pl.R) b[k] = dsin(th * float(k + 1)) * pre;
+      if (k < pl.R) b[k] = sk * pre;
       else b[k] = T(0.f);
+      T sn = c2 * sk - sp;
+      sp = sk;
+      sk = sn;
     }
   }
 }

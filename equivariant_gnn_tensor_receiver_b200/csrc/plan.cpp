@@ -16,6 +16,8 @@
 #include <vector>
 
 #include "plan.h"
+#include "pm_layout.h"
+#include "pf_layout.h"
 #include "workspace.h"
 
 using namespace tpc;
@@ -423,6 +425,40 @@ int tpconv_plan_create(tpconv_plan** out, const char* irreps_in, int l_sh_max,
         }
       }
     }
+  }
+  // path-major adjoint streams (all warps on one path at a time)
+  {
+    bool ok = true;
+    for (int i = 0; i < d.n_in; ++i) ok = ok && (d.in_mul[i] % 4 == 0);
+    for (int i = 0; i < d.n_out; ++i) ok = ok && (d.Kb[i] % 4 == 0);
+    d.pm_n3max = 1;
+    d.pm_n1max = 1;
+    for (int i = 0; i < P; ++i) {
+      d.pm_n3max = std::max(d.pm_n3max, 2 * int(d.path[i].l3) + 1);
+      d.pm_n1max = std::max(d.pm_n1max, 2 * int(d.path[i].l1) + 1);
+    }
+    auto pick = [&](bool dbl, int& tile, int& bytes) {
+      tile = 0;
+      bytes = 0;
+      const int cands[4] = {64, 32, 16, 8};
+      for (int t : cands) {
+        const int b = pm_smem_bytes(d.rm, t, d.pm_n3max, d.pm_n1max, R, dbl);
+        if (b <= 110 * 1024) {  // two CTAs per SM
+          tile = t;
+          bytes = b;
+          return;
+        }
+      }
+    };
+    pick(false, d.pm_tile_a, d.pm_smem_a);
+    pick(true, d.pm_tile_d, d.pm_smem_d);
+    d.pm_ok = ok && d.pm_tile_a > 0 && d.pm_tile_d > 0;
+    d.pf_nmz_max = 1;
+    for (int i = 0; i < P; ++i) d.pf_nmz_max = std::max(d.pf_nmz_max, int(d.path[i].nmz));
+    d.pf_smem_r = pf_smem_bytes(d.rm, d.pm_n1max, d.pf_nmz_max, false);
+    d.pf_smem_s = pf_smem_bytes(d.rm, d.pm_n3max, d.pf_nmz_max, false);
+    d.pf_smem_r2 = pf_smem_bytes(d.rm, d.pm_n1max, d.pf_nmz_max, true);
+    d.pf_smem_s2 = pf_smem_bytes(d.rm, d.pm_n3max, d.pf_nmz_max, true);
   }
   if (size_t(std::max(std::max(sm, sm2) * 4, std::max(d.fz_smem_f, d.fz_smem_s))) > 227 * 1024) {
     delete p;

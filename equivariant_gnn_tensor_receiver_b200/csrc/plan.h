@@ -122,6 +122,13 @@ struct DevPlan {
   int adj_cw;                       // adjoint stream channel tile (0: lane-per-edge stream unavailable)
   int adj_g, adj_xs, adj_smem;      // its G tile floats, staged row stride (odd), smem bytes
   int dadj_cw, dadj_g, dadj_xs, dadj_smem;  // the same for the double-backward adjoint stream
+  int pm_ok;                        // path-major adjoint streams usable (channel counts multiple of 4)
+  int pm_n3max, pm_n1max;           // largest 2l3+1 / 2l1+1 over the paths
+  int pm_tile_a, pm_smem_a;         // first-order path-major stream: channel tile, smem bytes
+  int pm_tile_d, pm_smem_d;         // second-order path-major stream: channel tile, smem bytes
+  int pf_nmz_max;                   // largest compact coupling matrix over the paths
+  int pf_smem_r, pf_smem_s;         // path-major node streams (receiver / sender form): smem bytes
+  int pf_smem_r2, pf_smem_s2;       // the same for their double-backward forms
   DevPath path[kMaxPaths];
 };
 

@@ -446,7 +446,7 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
       }
       {
         PhaseScope ps(TPCONV_PHASE_BWD_EDGE_R, s);
-        cudaError_t e = d.adj_cw > 0
+        cudaError_t e = d.pm_ok
                             ? TPC_RM_CALL(d.rm, launch_adj_rm, d, int(r0), nc, rowptr, col, edge_vec, x, S_, dvec, dY,
                                           db, s)
                             : TPC_RM_CALL(d.rm, launch_radj_rm, d, int(r0), nc, rowptr, col, edge_vec, x, S_, dvec,
@@ -553,7 +553,7 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
         }
       }
       PhaseScope ps(TPCONV_PHASE_DBL_EDGE_R, s);
-      cudaError_t e = d.dadj_cw > 0
+      cudaError_t e = d.pm_ok
                           ? TPC_RM_CALL(d.rm, launch_dadj_rm, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x,
                                         gg_x, G, has_t ? Gt : nullptr, d_vec, s)
                           : TPC_RM_CALL(d.rm, launch_dbl_r_rm, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x,

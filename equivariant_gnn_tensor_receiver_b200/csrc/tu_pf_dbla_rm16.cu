@@ -1,0 +1,7 @@
+// Path-major node stream (dbla form), radial width 16.
+#include "launch_pm.cuh"
+
+namespace tpc {
+template cudaError_t launch_dbl_a_rm<16>(const DevPlan&, int, int, const int*, const int*, const float*, const float*, const float*, const float*, float*, float*, cudaStream_t);
+}  // namespace tpc
+TPC_REGISTER_TU(pf_dbla_rm16, (&tpc::pf_smem_rm<16, true, true>))

@@ -1,0 +1,7 @@
+// Path-major node stream (send form), radial width 16.
+#include "launch_pm.cuh"
+
+namespace tpc {
+template cudaError_t launch_send_rm<16>(const DevPlan&, int, int, const int*, const int*, const int*, const float*, const float*, float*, cudaStream_t);
+}  // namespace tpc
+TPC_REGISTER_TU(pf_send_rm16, (&tpc::pf_smem_rm<16, false, false>))
