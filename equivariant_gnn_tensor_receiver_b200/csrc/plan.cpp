@@ -16,8 +16,7 @@
 #include <vector>
 
 #include "plan.h"
-#include "pm_layout.h"
-#include "pf_layout.h"
+#include "wn_layout.h"
 #include "workspace.h"
 
 using namespace tpc;
@@ -347,120 +346,46 @@ int tpconv_plan_create(tpconv_plan** out, const char* irreps_in, int l_sh_max,
   }
   d.sm_floats = sm;
   d.sm_floats2 = sm2;
-  // fused streams: all paths of a node in one CTA (one warp per path, passes of <= 14 warps)
+  // warp-per-node streams
   {
-    const int passes = (P + 13) / 14;
-    d.fz_warps = std::max(1, (P + passes - 1) / passes);
-    int msz = 0;
-    for (int i = 0; i < P; ++i) {
-      d.path[i].smf_off = msz;
-      msz += kEdgeBatch * ((d.path[i].nmz + 3) & ~3);
-    }
-    d.fz_cpl_f = d.max_c_in > 32 ? 2 : 1;
-    d.fz_cpl_s = d.max_c_out > 32 ? 2 : 1;
-    d.fz_xw_f = 0;
-    for (int i = 0; i < d.n_in; ++i) d.fz_xw_f += std::min(32 * d.fz_cpl_f, d.in_mul[i]) * (2 * d.in_l[i] + 1);
-    d.fz_xw_s = 0;
-    for (int i = 0; i < d.n_out; ++i) d.fz_xw_s += std::min(32 * d.fz_cpl_s, d.out_mul[i]) * (2 * d.out_l[i] + 1);
-    auto bytes = [&](int xw) {
-      int Y = 2 * kEdgeBatch * 16, B = 2 * kEdgeBatch * d.rm, S = 2 * kEdgeBatch, T = 2 * kMaxBlocks;
-      int X = (Y + B + S + T + 3) & ~3;
-      return (X + 2 * kEdgeBatch * xw + msz) * 4;
-    };
-    d.fz_smem_f = bytes(d.fz_xw_f);
-    d.fz_smem_s = bytes(d.fz_xw_s);
-  }
-  // lane-per-edge adjoint stream: channel tile cw (multiple of 4) chosen as large as fits
-  {
-    bool ok = true;
+    bool ok = true;  // 16-byte staging of rows and channel groups of four (adjoint streams)
     for (int i = 0; i < d.n_in; ++i) ok = ok && (d.in_mul[i] % 4 == 0);
     for (int i = 0; i < d.n_out; ++i) ok = ok && (d.Kb[i] % 4 == 0);
-    d.adj_cw = 0;
-    if (ok) {
-      int acc = 0, rn3 = 0;
-      for (int i = 0; i < P; ++i) {
-        d.path[i].adj_goff = rn3;
-        rn3 += R * (2 * d.path[i].l3 + 1);
-        d.path[i].adj_acc = acc;
-        acc += 32 * ((2 * d.path[i].l2 + 1) + d.rm);
-      }
-      const int cmax = (d.max_c_in + 3) & ~3;
-      const int cands[6] = {cmax, 128, 64, 32, 16, 4};
-      int dacc = 0;
-      for (int i = 0; i < P; ++i) {
-        d.path[i].dadj_acc = dacc;
-        dacc += 32 * (2 * (2 * d.path[i].l2 + 1) + 2 * d.rm);
-      }
-      d.dadj_cw = 0;
-      for (int c : cands) {
-        if (c > cmax || c <= 0) continue;
-        int xw = 0;
-        for (int i = 0; i < d.n_in; ++i) xw += std::min(c, d.in_mul[i]) * (2 * d.in_l[i] + 1);
-        const int xs = xw | 1;
-        const int g = rn3 * c;
-        const int head = 2 * g + 2 * 32 * xs + 2 * 32 * 16 + 2 * 32 * d.rm + 32;
-        const int bytes = (((head + 3) & ~3) + dacc) * 4;
-        if (bytes <= 227 * 1024) {
-          d.dadj_cw = c;
-          d.dadj_g = g;
-          d.dadj_xs = xs;
-          d.dadj_smem = bytes;
-          break;
-        }
-      }
-      for (int c : cands) {
-        if (c > cmax || c <= 0) continue;
-        int xw = 0;
-        for (int i = 0; i < d.n_in; ++i) xw += std::min(c, d.in_mul[i]) * (2 * d.in_l[i] + 1);
-        const int xs = xw | 1;
-        const int g = rn3 * c;
-        const int head = g + 32 * xs + 32 * 16 + 32 * d.rm + 32;
-        const int bytes = (((head + 3) & ~3) + acc) * 4;
-        if (bytes <= 227 * 1024) {
-          d.adj_cw = c;
-          d.adj_g = g;
-          d.adj_xs = xs;
-          d.adj_smem = bytes;
-          break;
-        }
-      }
-    }
-  }
-  // path-major adjoint streams (all warps on one path at a time)
-  {
-    bool ok = true;
-    for (int i = 0; i < d.n_in; ++i) ok = ok && (d.in_mul[i] % 4 == 0);
-    for (int i = 0; i < d.n_out; ++i) ok = ok && (d.Kb[i] % 4 == 0);
-    d.pm_n3max = 1;
-    d.pm_n1max = 1;
+    d.wn_ok = ok;
+    d.n3max = 1;
+    d.n1max = 1;
+    d.nmz_max = 1;
     for (int i = 0; i < P; ++i) {
-      d.pm_n3max = std::max(d.pm_n3max, 2 * int(d.path[i].l3) + 1);
-      d.pm_n1max = std::max(d.pm_n1max, 2 * int(d.path[i].l1) + 1);
+      d.n3max = std::max(d.n3max, 2 * int(d.path[i].l3) + 1);
+      d.n1max = std::max(d.n1max, 2 * int(d.path[i].l1) + 1);
+      d.nmz_max = std::max(d.nmz_max, int(d.path[i].nmz));
     }
-    auto pick = [&](bool dbl, int& tile, int& bytes) {
-      tile = 0;
-      bytes = 0;
-      const int cands[4] = {64, 32, 16, 8};
-      for (int t : cands) {
-        const int b = pm_smem_bytes(d.rm, t, d.pm_n3max, d.pm_n1max, R, dbl);
-        if (b <= 110 * 1024) {  // two CTAs per SM
-          tile = t;
-          bytes = b;
-          return;
-        }
-      }
-    };
-    pick(false, d.pm_tile_a, d.pm_smem_a);
-    pick(true, d.pm_tile_d, d.pm_smem_d);
-    d.pm_ok = ok && d.pm_tile_a > 0 && d.pm_tile_d > 0;
-    d.pf_nmz_max = 1;
-    for (int i = 0; i < P; ++i) d.pf_nmz_max = std::max(d.pf_nmz_max, int(d.path[i].nmz));
-    d.pf_smem_r = pf_smem_bytes(d.rm, d.pm_n1max, d.pf_nmz_max, false);
-    d.pf_smem_s = pf_smem_bytes(d.rm, d.pm_n3max, d.pf_nmz_max, false);
-    d.pf_smem_r2 = pf_smem_bytes(d.rm, d.pm_n1max, d.pf_nmz_max, true);
-    d.pf_smem_s2 = pf_smem_bytes(d.rm, d.pm_n3max, d.pf_nmz_max, true);
   }
-  if (size_t(std::max(std::max(sm, sm2) * 4, std::max(d.fz_smem_f, d.fz_smem_s))) > 227 * 1024) {
+  // warp-per-node streams: kernels instantiated for feature degrees <= 2 (radial
+  // width 8) or <= 3; two channels per lane when every path has >= 64 channels
+  {
+    int lmax = 0, cmin = 1 << 30;
+    for (int i = 0; i < P; ++i) {
+      lmax = std::max(lmax, std::max(int(d.path[i].l1), int(d.path[i].l3)));
+      cmin = std::min(cmin, std::min(d.path[i].c_in, d.path[i].c_out));
+    }
+    d.wn_lf = (d.rm == 8 && lmax <= 2) ? 2 : 3;
+    d.wn_cpl = (d.wn_lf == 2 && cmin >= 64) ? 2 : 1;
+    d.wn_smem_f = wn_smem_bytes(d.rm, d.wn_cpl, d.n1max, d.nmz_max, false, false);
+    d.wn_smem_s = wn_smem_bytes(d.rm, d.wn_cpl, d.n3max, d.nmz_max, false, false);
+    d.wn_smem_f2 = wn_smem_bytes(d.rm, 1, d.n1max, d.nmz_max, true, true);
+    d.wn_smem_s2 = wn_smem_bytes(d.rm, 1, d.n3max, d.nmz_max, true, false);
+    d.wn_smem_adj = wna_smem_bytes(d.rm, d.n3max, d.n1max, false);
+    d.wn_smem_dadj = wna_smem_bytes(d.rm, d.n3max, d.n1max, true);
+    const int mx = std::max(std::max(std::max(d.wn_smem_f, d.wn_smem_s), std::max(d.wn_smem_f2, d.wn_smem_s2)),
+                            std::max(d.wn_smem_adj, d.wn_smem_dadj));
+    if (mx > 227 * 1024) {
+      delete p;
+      return TPCONV_ERR_UNSUPPORTED;
+    }
+  }
+  // the per-path adjoint streams serve the plans whose rows cannot be staged 16 bytes at a time
+  if (!d.wn_ok && size_t(std::max(sm, sm2)) * 4 > 227 * 1024) {
     delete p;
     return TPCONV_ERR_UNSUPPORTED;
   }

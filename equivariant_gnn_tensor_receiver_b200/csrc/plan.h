@@ -92,12 +92,8 @@ struct DevPath {
   int32_t kxoff;            // B column of (k=0, w=0) in input block i1: kxoff + k*c_out + w
   int64_t theta_off;        // start of Theta[p] ([R][c_in][c_out])
   int32_t nmz;              // m_count(l1, l2, l3)
-  int32_t sm_off;           // float offset of this path's warp scratch (first-order adjoint stream)
-  int32_t sm_off2;          // same for the double-backward adjoint stream
-  int32_t smf_off;          // float offset of this path's coupling-matrix scratch in the fused streams
-  int32_t adj_goff;         // adjoint stream: this path's G tile at adj_goff * channel-tile floats
-  int32_t adj_acc;          // adjoint stream: float offset of this path's per-edge partials
-  int32_t dadj_acc;         // double-backward adjoint stream: same
+  int32_t sm_off;           // float offset of this path's warp scratch (per-path adjoint stream)
+  int32_t sm_off2;          // same for the per-path double-backward adjoint stream
 };
 
 struct DevPlan {
@@ -113,22 +109,16 @@ struct DevPlan {
   int64_t b_pref[kMaxBlocks + 1];   // floats per node before block i1 (sum n1 * Kx)
   int max_c_in, max_c_out;
   int rm;                           // radial registers per lane (4, 8 or 16) >= R
-  int sm_floats;                    // dynamic smem floats of the first-order adjoint stream
-  int sm_floats2;                   // dynamic smem floats of the double-backward adjoint stream
-  int fz_warps;                     // warps per CTA of the fused streams (paths run in passes)
-  int fz_cpl_f, fz_xw_f;            // forward: channels per lane, staged x floats per edge
-  int fz_cpl_s, fz_xw_s;            // sender stream: channels per lane, staged g floats per edge
-  int fz_smem_f, fz_smem_s;         // dynamic smem bytes of the fused forward / sender streams
-  int adj_cw;                       // adjoint stream channel tile (0: lane-per-edge stream unavailable)
-  int adj_g, adj_xs, adj_smem;      // its G tile floats, staged row stride (odd), smem bytes
-  int dadj_cw, dadj_g, dadj_xs, dadj_smem;  // the same for the double-backward adjoint stream
-  int pm_ok;                        // path-major adjoint streams usable (channel counts multiple of 4)
-  int pm_n3max, pm_n1max;           // largest 2l3+1 / 2l1+1 over the paths
-  int pm_tile_a, pm_smem_a;         // first-order path-major stream: channel tile, smem bytes
-  int pm_tile_d, pm_smem_d;         // second-order path-major stream: channel tile, smem bytes
-  int pf_nmz_max;                   // largest compact coupling matrix over the paths
-  int pf_smem_r, pf_smem_s;         // path-major node streams (receiver / sender form): smem bytes
-  int pf_smem_r2, pf_smem_s2;       // the same for their double-backward forms
+  int sm_floats;                    // dynamic smem floats of the per-path adjoint stream
+  int sm_floats2;                   // the same for its double-backward form
+  int wn_ok;                        // rows stageable 16 bytes at a time (channel counts multiple of 4)
+  int n3max, n1max;                 // largest 2l3+1 / 2l1+1 over the paths
+  int nmz_max;                      // largest compact coupling matrix over the paths
+  int wn_lf;                        // warp-per-node streams: bound on l1, l3 of the instantiation (2 or 3)
+  int wn_cpl;                       // channels per lane of their first-order channel-lane forms (1 or 2)
+  int wn_smem_f, wn_smem_s;         // dynamic smem bytes: receiver / sender form, first order
+  int wn_smem_f2, wn_smem_s2;       // the same, second order
+  int wn_smem_adj, wn_smem_dadj;    // receiver adjoint streams, first / second order
   DevPath path[kMaxPaths];
 };
 

@@ -365,22 +365,26 @@ __device__ __forceinline__ void edge_vec_grad2(const DevPlan& pl, const float* v
   }
   DD nx, ny, nz, r;
   unit(c[0], c[1], c[2], nx, ny, nz, r);
-  DD Y[16];
-  switch (pl.lsh) {
-    case 0: sh_all<0>(nx, ny, nz, Y); break;
-    case 1: sh_all<1>(nx, ny, nz, Y); break;
-    case 2: sh_all<2>(nx, ny, nz, Y); break;
-    default: sh_all<3>(nx, ny, nz, Y); break;
-  }
+  float g[3] = {0.f, 0.f, 0.f};
+  // one SH degree at a time keeps the nested duals of only 2l+1 harmonics live
+  auto degree = [&](auto LC) {
+    constexpr int L = decltype(LC)::value;
+    if (L > pl.lsh) return;
+    DD Y[2 * L + 1];
+    sh_degree<L>(nx, ny, nz, Y);
+#pragma unroll
+    for (int i = 0; i < 2 * L + 1; ++i) {
+      const int m = L * L + i;
+#pragma unroll
+      for (int a = 0; a < 3; ++a) g[a] = fmaf(wY[m], Y[i].d[a].v, fmaf(hY[m], Y[i].d[a].d[0], g[a]));
+    }
+  };
+  degree(std::integral_constant<int, 0>{});
+  degree(std::integral_constant<int, 1>{});
+  degree(std::integral_constant<int, 2>{});
+  degree(std::integral_constant<int, 3>{});
   DD b[RM];
   radial_basis<RM>(pl, r, b);
-  float g[3] = {0.f, 0.f, 0.f};
-#pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    if (m >= pl.n_sh) break;
-#pragma unroll
-    for (int i = 0; i < 3; ++i) g[i] = fmaf(wY[m], Y[m].d[i].v, fmaf(hY[m], Y[m].d[i].d[0], g[i]));
-  }
 #pragma unroll
   for (int k = 0; k < RM; ++k) {
     if (k >= pl.R) break;

@@ -1,0 +1,283 @@
+// Warp-per-node edge streams, lane = channel (receiver and sender forms, first
+// and second order).
+//
+// One warp owns one node of the chunk and walks its CSR segment once per path
+// and channel tile.  Lane j computes the geometry of edge j of each 32-edge
+// batch (unit vector, spherical harmonics of the path's degree l2, radial basis)
+// and the edge's compact coupling matrix M[m1][m3] = sum_m2 C[m1,m2,m3] Y[m2];
+// both go to the warp's shared slice and are read back by every lane with
+// broadcast 16-byte loads.  The neighbours' feature rows are staged by cp.async
+// in sub-batches of kWnSub edges, double-buffered, so the gather of the next
+// sub-batch overlaps the FFMA work of the current one.  Lane u keeps the node's
+// partial state for its CPL channels in registers over the whole segment and
+// writes it once: no block barrier, no cross-warp reduction, no atomics.
+//
+// Forms (streaming schedule of "Sobek", arXiv 2607.18074, abstract: edge-local
+// products consumed directly into bounded node-side state):
+//   receiver, first order   A[r,k,u,m3]  = sum_e b_ek (M_e x_s[u])[m3]
+//   sender,   first order   B[s,k,w,m1]  = sum_e b_ek (M_e^T g_r[w])[m1]
+//   receiver, second order  A1 = sum_e b (M x1 + Md x) + bd (M x),  A0 = sum_e b (M x)
+//   sender,   second order  B1 = sum_e b (Md^T g) + bd (M^T g),     B0 = sum_e b (M^T g)
+// where Md, bd are the derivatives of M_e, b_e along the edge-vector
+// perturbation gg_vec_e and x1 = gg_x (terms with a missing input are zero).
+#pragma once
+
+#include "async_copy.cuh"
+#include "streams.cuh"
+#include "wn_layout.h"
+
+namespace tpc {
+
+// Geometry of edge e for one path: Y of degree L2 and the radial basis (and,
+// when DIR, their derivatives along the perturbation ggv_e of the edge vector).
+template <int L2, int RM, bool DIR>
+__device__ __forceinline__ void wn_geometry(const DevPlan& pl, const float* __restrict__ vec,
+                                            const float* __restrict__ ggv, int e, float* Y, float* Yd, float* b,
+                                            float* bd) {
+  constexpr int N2 = 2 * L2 + 1;
+  if constexpr (!DIR) {
+    const float vx = vec[3 * e], vy = vec[3 * e + 1], vz = vec[3 * e + 2];
+    float nx, ny, nz, r;
+    unit(vx, vy, vz, nx, ny, nz, r);
+    sh_degree<L2>(nx, ny, nz, Y);
+    radial_basis<RM>(pl, r, b);
+  } else {
+    using D1 = Dual<float, 1>;
+    D1 vx(vec[3 * e]), vy(vec[3 * e + 1]), vz(vec[3 * e + 2]);
+    if (ggv) {
+      vx.d[0] = ggv[3 * e];
+      vy.d[0] = ggv[3 * e + 1];
+      vz.d[0] = ggv[3 * e + 2];
+    }
+    D1 nx, ny, nz, r;
+    unit(vx, vy, vz, nx, ny, nz, r);
+    D1 Yv[N2], bv[RM];
+    sh_degree<L2>(nx, ny, nz, Yv);
+    radial_basis<RM>(pl, r, bv);
+#pragma unroll
+    for (int i = 0; i < N2; ++i) {
+      Y[i] = Yv[i].v;
+      Yd[i] = Yv[i].d[0];
+    }
+#pragma unroll
+    for (int k = 0; k < RM; ++k) {
+      b[k] = bv[k].v;
+      bd[k] = bv[k].d[0];
+    }
+  }
+}
+
+// compact coupling matrix of one edge, padded with zeros to NMP entries
+template <int L1, int L2, int L3, int NMP>
+__device__ __forceinline__ void wn_coupling(const float* Y, float* Mrow) {
+  constexpr int NMZ = Tri<L1, L2, L3>::NMZ;
+  coupling_row<L1, L2, L3>(Y, Mrow);
+#pragma unroll
+  for (int i = NMZ; i < NMP; ++i) Mrow[i] = 0.f;
+}
+
+// one path, all channel tiles of the warp's node
+template <int L1, int L2, int L3, int RM, int CPL, bool RECV, bool DBL>
+__device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q, const WnLay& L, float* ws, int nl,
+                                             int nc, int a0, int a1, const int* __restrict__ nbr,
+                                             const int* __restrict__ perm, const float* __restrict__ vec,
+                                             const float* __restrict__ ggv, const float* __restrict__ src,
+                                             const float* __restrict__ src1, float* __restrict__ out,
+                                             float* __restrict__ out0) {
+  using TR = Tri<L1, L2, L3>;
+  constexpr int N2 = TR::N2, NMZ = TR::NMZ, NMP = (NMZ + 3) & ~3;
+  constexpr int NI = RECV ? TR::N1 : TR::N3;  // staged floats per channel
+  constexpr int NO = RECV ? TR::N3 : TR::N1;  // state floats per channel and radial index
+  constexpr int NPART = DBL ? 2 : 1;
+  constexpr int NACC = NPART * CPL * RM * NO;
+  const int lane = lane_id();
+  const int c = RECV ? q.c_in : q.c_out;
+  const int dim = RECV ? pl.dim_in : pl.dim_out;
+  const int off = RECV ? q.in_off : q.out_off;
+  const int ne = a1 - a0;
+  const int nsb = (ne + kWnSub - 1) / kWnSub;
+  const bool two = DBL && RECV && src1 != nullptr;
+  float* sM = ws + L.M;
+  float* sMd = ws + L.Md;
+  float* sB = ws + L.B;
+  float* sBd = ws + L.Bd;
+
+  for (int c0 = 0; c0 < c; c0 += 32 * CPL) {
+    const int w = min(32 * CPL, c - c0);
+    const int len = w * NI;
+    const bool v4 = ((dim | off | len) & 3) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0 &&
+                    (reinterpret_cast<uintptr_t>(src1) & 15) == 0;
+    const size_t coff = size_t(off) + size_t(c0) * NI;
+    // stage the rows of sub-batch sb into buffer sb & 1 (one commit group per call site)
+    auto stage = [&](int sb) {
+      const int j0 = sb * kWnSub, nb = min(kWnSub, ne - j0);
+      float* X = ws + L.X + (sb & 1) * L.buf;
+      float* X1 = ws + L.X1 + (sb & 1) * L.buf;
+      for (int j = 0; j < nb; ++j) {
+        const size_t row = size_t(nbr[a0 + j0 + j]) * dim + coff;
+        if (v4) {
+          for (int o = 4 * lane; o < len; o += 128) {
+            ac_copy16(X + j * L.xs + o, src + row + o);
+            if (two) ac_copy16(X1 + j * L.xs + o, src1 + row + o);
+          }
+        } else {
+          for (int o = lane; o < len; o += 32) {
+            ac_copy4(X + j * L.xs + o, src + row + o);
+            if (two) ac_copy4(X1 + j * L.xs + o, src1 + row + o);
+          }
+        }
+      }
+    };
+
+    float acc[NACC];
+#pragma unroll
+    for (int i = 0; i < NACC; ++i) acc[i] = 0.f;
+
+    if (nsb > 0) stage(0);
+    ac_commit();
+    for (int sb = 0; sb < nsb; ++sb) {
+      const int j0 = sb * kWnSub;
+      if ((j0 & 31) == 0) {
+        // geometry and coupling matrices of the next 32 edges, lane = edge
+        __syncwarp();
+        const int j = j0 + lane;
+        if (j < ne) {
+          const int e = RECV ? a0 + j : perm[a0 + j];
+          float Y[N2], Yd[N2], b[RM], bd[RM], Mrow[NMP];
+          wn_geometry<L2, RM, DBL>(pl, vec, ggv, e, Y, Yd, b, bd);
+          wn_coupling<L1, L2, L3, NMP>(Y, Mrow);
+          sts_vec<NMP>(sM + lane * L.nmp, Mrow);
+          sts_vec<RM>(sB + lane * RM, b);
+          if constexpr (DBL) {
+            wn_coupling<L1, L2, L3, NMP>(Yd, Mrow);
+            sts_vec<NMP>(sMd + lane * L.nmp, Mrow);
+            sts_vec<RM>(sBd + lane * RM, bd);
+          }
+        }
+        __syncwarp();
+      }
+      if (sb + 1 < nsb) stage(sb + 1);
+      ac_commit();
+      ac_wait<1>();
+      __syncwarp();
+      const float* X = ws + L.X + (sb & 1) * L.buf;
+      const float* X1 = ws + L.X1 + (sb & 1) * L.buf;
+      const int nb = min(kWnSub, ne - j0);
+      for (int jj = 0; jj < nb; ++jj) {
+        const int js = (j0 & 31) + jj;
+        float Mv[NMP], bv[RM];
+        lds_vec<NMP>(sM + js * L.nmp, Mv);
+        lds_vec<RM>(sB + js * RM, bv);
+        float Mdv[DBL ? NMP : 1], bdv[DBL ? RM : 1];
+        if constexpr (DBL) {
+          lds_vec<NMP>(sMd + js * L.nmp, Mdv);
+          lds_vec<RM>(sBd + js * RM, bdv);
+        }
+#pragma unroll
+        for (int h = 0; h < CPL; ++h) {
+          const int cb = jj * L.xs + (lane + 32 * h) * NI;
+          float xv[NI];
+#pragma unroll
+          for (int i = 0; i < NI; ++i) xv[i] = X[cb + i];
+          float* a = acc + h * RM * NO;                  // part 0
+          float* a1 = acc + (CPL + h) * RM * NO;         // part 1 (second order)
+          if constexpr (!DBL) {
+            float T[NO];
+            if constexpr (RECV) apply_M<L1, L2, L3>(Mv, xv, T);
+            else apply_Mt<L1, L2, L3>(Mv, xv, T);
+#pragma unroll
+            for (int k = 0; k < RM; ++k)
+#pragma unroll
+              for (int i = 0; i < NO; ++i) a[k * NO + i] = fmaf(bv[k], T[i], a[k * NO + i]);
+          } else if constexpr (RECV) {
+            float x1v[NI], T[NO], T1[NO], T2[NO];
+#pragma unroll
+            for (int i = 0; i < NI; ++i) x1v[i] = two ? X1[cb + i] : 0.f;
+            apply_M<L1, L2, L3>(Mv, xv, T);
+            apply_M<L1, L2, L3>(Mv, x1v, T1);
+            apply_M<L1, L2, L3>(Mdv, xv, T2);
+#pragma unroll
+            for (int i = 0; i < NO; ++i) T1[i] += T2[i];
+#pragma unroll
+            for (int k = 0; k < RM; ++k)
+#pragma unroll
+              for (int i = 0; i < NO; ++i) {
+                a[k * NO + i] = fmaf(bv[k], T1[i], fmaf(bdv[k], T[i], a[k * NO + i]));
+                a1[k * NO + i] = fmaf(bv[k], T[i], a1[k * NO + i]);
+              }
+          } else {
+            float U[NO], U1[NO];
+            apply_Mt<L1, L2, L3>(Mv, xv, U);
+            apply_Mt<L1, L2, L3>(Mdv, xv, U1);
+#pragma unroll
+            for (int k = 0; k < RM; ++k)
+#pragma unroll
+              for (int i = 0; i < NO; ++i) {
+                a[k * NO + i] = fmaf(bv[k], U1[i], fmaf(bdv[k], U[i], a[k * NO + i]));
+                a1[k * NO + i] = fmaf(bv[k], U[i], a1[k * NO + i]);
+              }
+          }
+        }
+      }
+      __syncwarp();
+    }
+
+    // node state rows: A block i3 (B block i1), row nl * NO + i, column koff + k * c + channel
+    const int Kq = RECV ? pl.Kb[q.i3] : pl.Kx[q.i1];
+    const int64_t pref = RECV ? pl.a_pref[q.i3] : pl.b_pref[q.i1];
+    const size_t base = size_t(nc) * pref + size_t(nl) * NO * Kq + (RECV ? q.koff : q.kxoff) + c0;
+#pragma unroll
+    for (int part = 0; part < NPART; ++part) {
+      float* dst = part == 0 ? out : out0;
+#pragma unroll
+      for (int h = 0; h < CPL; ++h) {
+        const int ch = lane + 32 * h;
+        if (ch >= w) continue;
+#pragma unroll
+        for (int k = 0; k < RM; ++k) {
+          if (k >= pl.R) break;
+#pragma unroll
+          for (int i = 0; i < NO; ++i)
+            dst[base + size_t(i) * Kq + k * c + ch] = acc[((part * CPL + h) * RM + k) * NO + i];
+        }
+      }
+    }
+  }
+}
+
+// grid: P * ceil(nc / kWnWarps) CTAs of kWnWarps warps, path-major: CTA b runs
+// path b / nblk for nodes n0 + (b % nblk) * kWnWarps + warp.  CTAs are dispatched
+// roughly in index order, so the CTAs resident at any time run one or two path
+// bodies and share their instructions in the instruction caches.
+// RECV: ptr = rowptr, nbr = col (edge id = CSR position); else ptr = s_rowptr,
+// nbr = s_recv, perm = sender-sorted position -> edge id.
+template <int RM, int LF, int CPL, bool RECV, bool DBL>
+__global__ void __launch_bounds__(32 * kWnWarps, 3)
+    k_wn_stream(const __grid_constant__ DevPlan pl, int n0, int nc, const int* __restrict__ ptr,
+                const int* __restrict__ nbr, const int* __restrict__ perm, const float* __restrict__ vec,
+                const float* __restrict__ ggv, const float* __restrict__ src, const float* __restrict__ src1,
+                float* __restrict__ out, float* __restrict__ out0) {
+  extern __shared__ __align__(16) float sm[];
+  const int warp = threadIdx.x >> 5;
+  const int nblk = (nc + kWnWarps - 1) / kWnWarps;
+  const int p = blockIdx.x / nblk;
+  const int nl = (blockIdx.x - p * nblk) * kWnWarps + warp;
+  if (nl >= nc) return;
+  const WnLay L = wn_layout_of(RM, CPL, RECV ? pl.n1max : pl.n3max, pl.nmz_max, DBL, DBL && RECV);
+  float* ws = sm + warp * L.total;
+  const int a0 = ptr[n0 + nl], a1 = ptr[n0 + nl + 1];
+  const DevPath& q = pl.path[p];
+  switch (triple_id(q.l1, q.l2, q.l3)) {
+#define TPC_CASE(a, b, c)                                                                                        \
+  case triple_id(a, b, c):                                                                                       \
+    if constexpr (a <= LF && c <= LF)                                                                            \
+      wn_chan_path<a, b, c, RM, CPL, RECV, DBL>(pl, q, L, ws, nl, nc, a0, a1, nbr, perm, vec, ggv, src, src1, out, \
+                                                out0);                                                           \
+    break;
+    TPC_FOR_EACH_TRIPLE(TPC_CASE)
+#undef TPC_CASE
+    default: break;
+  }
+}
+
+}  // namespace tpc

@@ -1,0 +1,346 @@
+// Warp-per-node receiver adjoint streams, lane = edge (first and second order).
+//
+// One warp owns one receiver r and walks its CSR segment in batches of 32
+// edges, one edge per lane.  The node-side adjoint state G = Theta^T g_r (and,
+// for the double backward, Gt = gg_Theta^T g_r) is staged by cp.async in chunks
+// of kWnChunk channels as [u][k][m3], so that every lane reads a channel's
+// RM x n3 block with broadcast 16-byte loads, while each lane stages and reads
+// its own edge's sender row.  All reductions over channels happen in the lane's
+// registers; the CG contraction with the per-edge outer-product accumulator Q
+// runs once per path rather than once per channel.
+//
+// First order (e = s -> r):
+//     db_ek = sum_{p,u,m3} G[k,p,u,m3] (M_e x_s[u])[m3]
+//     dY_e  = sum_p C_p : Q_p,   Q_p[m1][m3] = sum_u x_s[u,m1] (sum_k b_ek G[k,p,u,m3])
+//     dvec_e = J_Y^T dY_e + J_b^T db_e
+// Second order (Md, bd along gg_vec_e, x1 = gg_x), per channel:
+//     dG = sum_k b_k G_k,  dX = sum_k (b_k Gt_k + bd_k G_k),  T0 = M x,  T12 = M x1 + Md x
+//     wb_k += G_k.T12 + Gt_k.T0,  hb_k += G_k.T0
+//     Qw += x1 (x) dG + x (x) dX,  Qh += x (x) dG
+//     d_vec_e = grad_v [wY.Y + hY.Ydot + wb.b + hb.bdot],  wY = C:Qw, hY = C:Qh
+// Backward of the streaming schedule ("Sobek", arXiv 2607.18074, abstract).
+#pragma once
+
+#include "async_copy.cuh"
+#include "streams_dbl.cuh"
+#include "wn_layout.h"
+
+namespace tpc {
+
+// Q[m1][m3] += a[m1] c[m3] on the structural nonzeros of the coupling matrix
+template <int L1, int L2, int L3>
+__device__ __forceinline__ void outer_Q(const float* a, const float* c, float* Q) {
+  using TR = Tri<L1, L2, L3>;
+  sfor<TR::N1>([&](auto I1) {
+    sfor<TR::N3>([&](auto I3) {
+      constexpr int i1 = decltype(I1)::value, i3 = decltype(I3)::value;
+      if constexpr (TR::tab.m[i1][i3]) {
+        constexpr int mi = TR::tab.mi[i1][i3];
+        Q[mi] = fmaf(a[i1], c[i3], Q[mi]);
+      }
+    });
+  });
+}
+
+// out[m2] += sum_{m1,m3} C[m1,m2,m3] Q[m1][m3]
+template <int L1, int L2, int L3>
+__device__ __forceinline__ void contract_Q(const float* Q, float* out) {
+  using TR = Tri<L1, L2, L3>;
+  sfor<TR::N1>([&](auto I1) {
+    sfor<TR::N3>([&](auto I3) {
+      constexpr int i1 = decltype(I1)::value, i3 = decltype(I3)::value;
+      if constexpr (TR::tab.m[i1][i3]) {
+        constexpr int mi = TR::tab.mi[i1][i3];
+        sfor<TR::N2>([&](auto I2) {
+          constexpr int i2 = decltype(I2)::value;
+          if constexpr (TR::tab.cg[i1][i2][i3]) out[i2] = fmaf(TR::template cg<i1, i2, i3>(), Q[mi], out[i2]);
+        });
+      }
+    });
+  });
+}
+
+// one path of one 32-edge batch
+template <int L1, int L2, int L3, int RM, bool DBL>
+__device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, const WnaLay& L, float* ws, int rl,
+                                         int nc, int nb, int myrow, const float* __restrict__ x,
+                                         const float* __restrict__ x1, const float* __restrict__ G,
+                                         const float* __restrict__ Gt, float* db, float* hb) {
+  using TR = Tri<L1, L2, L3>;
+  constexpr int N1 = TR::N1, N2 = TR::N2, N3 = TR::N3, NMZ = TR::NMZ, GW = RM * N3;
+  constexpr int CH = kWnChunk;
+  static_assert(CH == 4, "the chunk is one group of four channels");
+  const int lane = lane_id();
+  const float* geo = ws + L.Geo + lane * L.geos;
+  float Mv[NMZ], bv[RM];
+  {
+    float Y[N2];
+#pragma unroll
+    for (int i = 0; i < N2; ++i) Y[i] = geo[L2 * L2 + i];
+    coupling_row<L1, L2, L3>(Y, Mv);
+#pragma unroll
+    for (int k = 0; k < RM; ++k) bv[k] = geo[16 + k];
+  }
+  float Mdv[DBL ? NMZ : 1], bdv[DBL ? RM : 1];
+  if constexpr (DBL) {
+    float Y[N2];
+#pragma unroll
+    for (int i = 0; i < N2; ++i) Y[i] = geo[16 + RM + L2 * L2 + i];
+    coupling_row<L1, L2, L3>(Y, Mdv);
+#pragma unroll
+    for (int k = 0; k < RM; ++k) bdv[k] = geo[32 + RM + k];
+  }
+  float Q[NMZ], Qh[DBL ? NMZ : 1];
+#pragma unroll
+  for (int i = 0; i < NMZ; ++i) Q[i] = 0.f;
+  if constexpr (DBL) {
+#pragma unroll
+    for (int i = 0; i < NMZ; ++i) Qh[i] = 0.f;
+  }
+
+  const int c = q.c_in, R = pl.R;
+  const int nch = c / CH;  // channel counts are multiples of four on this path
+  const int Kb = pl.Kb[q.i3];
+  const size_t gbase = size_t(nc) * pl.a_pref[q.i3] + size_t(rl) * N3 * Kb + q.koff;
+  const bool has_t = DBL && Gt != nullptr, has_x1 = DBL && x1 != nullptr;
+  auto stage = [&](int ch) {
+    const int u0 = ch * CH;
+    float* sG = ws + L.G + (ch & 1) * L.gbuf;
+    float* sGt = ws + L.Gt + (ch & 1) * L.gbuf;
+    for (int t = lane; t < R * N3 * CH; t += 32) {
+      const int u = t & (CH - 1), km = t / CH;  // km = k * N3 + m3
+      const int k = km / N3, m3 = km - k * N3;
+      const size_t src = gbase + size_t(m3) * Kb + size_t(k) * c + u0 + u;
+      ac_copy4(sG + u * L.gs + km, G + src);
+      if (has_t) ac_copy4(sGt + u * L.gs + km, Gt + src);
+    }
+    // the batch's rows, N1 16-byte pieces each, copied by the whole warp (coalesced)
+    float* sX = ws + L.X + (ch & 1) * L.xbuf;
+    float* sX1 = ws + L.X1 + (ch & 1) * L.xbuf;
+    const size_t cofs = size_t(q.in_off) + size_t(u0) * N1;
+#pragma unroll
+    for (int it = 0; it < N1; ++it) {
+      const int qd = it * 32 + lane;
+      const int j = qd / N1, v = qd - j * N1;
+      const int rj = __shfl_sync(0xffffffffu, myrow, j);
+      if (j < nb) {
+        const size_t src = size_t(rj) * pl.dim_in + cofs + 4 * v;
+        ac_copy16(sX + j * L.xs + 4 * v, x + src);
+        if (has_x1) ac_copy16(sX1 + j * L.xs + 4 * v, x1 + src);
+      }
+    }
+  };
+
+  if (nch > 0) stage(0);
+  ac_commit();
+  for (int ch = 0; ch < nch; ++ch) {
+    if (ch + 1 < nch) stage(ch + 1);
+    ac_commit();
+    ac_wait<1>();
+    __syncwarp();
+    const float* sG = ws + L.G + (ch & 1) * L.gbuf;
+    const float* sGt = ws + L.Gt + (ch & 1) * L.gbuf;
+    // the lane's four channels in N1 16-byte reads
+    float xg[CH * N1], x1g[DBL ? CH * N1 : 1];
+    lds_vec<CH * N1>(ws + L.X + (ch & 1) * L.xbuf + lane * L.xs, xg);
+    if constexpr (DBL) lds_vec<CH * N1>(ws + L.X1 + (ch & 1) * L.xbuf + lane * L.xs, x1g);
+#pragma unroll
+    for (int t = 0; t < CH; ++t) {
+      const float* xv = xg + t * N1;
+      const float* x1v = DBL ? x1g + t * N1 : xv;
+      float T[N3];
+      apply_M<L1, L2, L3>(Mv, xv, T);
+      if constexpr (!DBL) {
+        float g[GW];
+        lds_vec<GW>(sG + t * L.gs, g);
+        float dT[N3];
+#pragma unroll
+        for (int i = 0; i < N3; ++i) dT[i] = 0.f;
+#pragma unroll
+        for (int k = 0; k < RM; ++k) {
+          float s = 0.f;
+#pragma unroll
+          for (int i = 0; i < N3; ++i) {
+            dT[i] = fmaf(bv[k], g[k * N3 + i], dT[i]);
+            s = fmaf(g[k * N3 + i], T[i], s);
+          }
+          db[k] += s;
+        }
+        outer_Q<L1, L2, L3>(xv, dT, Q);
+      } else {
+        float T12[N3], Tb[N3];
+        apply_M<L1, L2, L3>(Mv, x1v, T12);
+        apply_M<L1, L2, L3>(Mdv, xv, Tb);
+#pragma unroll
+        for (int i = 0; i < N3; ++i) T12[i] += Tb[i];
+        float dG[N3], dX[N3];
+#pragma unroll
+        for (int i = 0; i < N3; ++i) dG[i] = dX[i] = 0.f;
+        // G and Gt rows in KH slices of RM / KH radial indices (bounds the live registers)
+        constexpr int KH = RM >= 8 ? 2 : 1, KS = RM / KH;
+#pragma unroll
+        for (int kh = 0; kh < KH; ++kh) {
+          float g[KS * N3], gt[KS * N3];
+          lds_vec<KS * N3>(sG + t * L.gs + kh * KS * N3, g);
+          lds_vec<KS * N3>(sGt + t * L.gs + kh * KS * N3, gt);
+#pragma unroll
+          for (int kk = 0; kk < KS; ++kk) {
+            const int k = kh * KS + kk;
+            float s1 = 0.f, s0 = 0.f;
+#pragma unroll
+            for (int i = 0; i < N3; ++i) {
+              const float gv = g[kk * N3 + i], tv = gt[kk * N3 + i];
+              dG[i] = fmaf(bv[k], gv, dG[i]);
+              dX[i] = fmaf(bv[k], tv, fmaf(bdv[k], gv, dX[i]));
+              s1 = fmaf(gv, T12[i], fmaf(tv, T[i], s1));
+              s0 = fmaf(gv, T[i], s0);
+            }
+            db[k] += s1;
+            hb[k] += s0;
+          }
+        }
+        outer_Q<L1, L2, L3>(x1v, dG, Q);
+        outer_Q<L1, L2, L3>(xv, dX, Q);
+        outer_Q<L1, L2, L3>(xv, dG, Qh);
+      }
+    }
+    __syncwarp();
+  }
+  // this path's share of dY (second order: wY, hY) for the lane's edge
+  float* acc = ws + L.Acc + lane * L.accs;
+  float o[N2];
+#pragma unroll
+  for (int i = 0; i < N2; ++i) o[i] = 0.f;
+  contract_Q<L1, L2, L3>(Q, o);
+#pragma unroll
+  for (int i = 0; i < N2; ++i) acc[L2 * L2 + i] += o[i];
+  if constexpr (DBL) {
+#pragma unroll
+    for (int i = 0; i < N2; ++i) o[i] = 0.f;
+    contract_Q<L1, L2, L3>(Qh, o);
+#pragma unroll
+    for (int i = 0; i < N2; ++i) acc[16 + L2 * L2 + i] += o[i];
+  }
+}
+
+// grid: ceil(nc / kWnWarps) CTAs of kWnWarps warps; warp = receiver r0 + rl.
+// The warps of a CTA step through the paths together (one barrier per path), so
+// that the resident warps of an SM share one or two path bodies in the
+// instruction caches; every warp runs the CTA's largest batch count, the ones
+// with fewer batches (or no node) joining the barriers without work.
+// First order writes dvec (and, when given, dY [E][n_sh], db [E][R]); second
+// order writes dvec.  x1 / Gt / ggv may be null (their terms vanish).
+template <int RM, int LF, bool DBL>
+__global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
+    k_wn_adj(const __grid_constant__ DevPlan pl, int r0, int nc, const int* __restrict__ rowptr,
+             const int* __restrict__ col, const float* __restrict__ vec, const float* __restrict__ ggv,
+             const float* __restrict__ x, const float* __restrict__ x1, const float* __restrict__ G,
+             const float* __restrict__ Gt, float* __restrict__ dvec, float* __restrict__ dYout,
+             float* __restrict__ dbout) {
+  extern __shared__ __align__(16) float sm[];
+  const int warp = threadIdx.x >> 5, lane = lane_id();
+  const int rl = blockIdx.x * kWnWarps + warp;
+  const bool has_node = rl < nc;
+  const WnaLay L = wna_layout_of(RM, pl.n3max, pl.n1max, DBL);
+  int& s_nbat = *reinterpret_cast<int*>(sm + kWnWarps * L.total);  // CTA batch count
+  float* ws = sm + warp * L.total;
+  // staged buffers read where nothing was staged must hold zeros
+  for (int i = lane; i < L.Geo; i += 32) ws[i] = 0.f;
+  const int e0 = has_node ? rowptr[r0 + rl] : 0, e1 = has_node ? rowptr[r0 + rl + 1] : 0;
+  if (threadIdx.x == 0) s_nbat = 0;
+  __syncthreads();
+  if (lane == 0 && e1 > e0) atomicMax(&s_nbat, (e1 - e0 + 31) / 32);
+  __syncthreads();
+  const int nbat = s_nbat;
+  for (int bi = 0; bi < nbat; ++bi) {
+    const int eb = e0 + 32 * bi;
+    const int nb = max(0, min(32, e1 - eb));
+    const bool valid = lane < nb;
+    const int e = eb + lane;
+    int myrow = 0;
+    float* geo = ws + L.Geo + lane * L.geos;
+    float* acc = ws + L.Acc + lane * L.accs;
+    if (valid) {
+      myrow = col[e];
+      using D1 = Dual<float, 1>;
+      D1 vx(vec[3 * e]), vy(vec[3 * e + 1]), vz(vec[3 * e + 2]);
+      if (DBL && ggv) {
+        vx.d[0] = ggv[3 * e];
+        vy.d[0] = ggv[3 * e + 1];
+        vz.d[0] = ggv[3 * e + 2];
+      }
+      D1 nx, ny, nz, rr;
+      unit(vx, vy, vz, nx, ny, nz, rr);
+      D1 Y[16], b[RM];
+#pragma unroll
+      for (int m = 0; m < 16; ++m) Y[m] = D1(0.f);
+      switch (pl.lsh) {
+        case 0: sh_all<0>(nx, ny, nz, Y); break;
+        case 1: sh_all<1>(nx, ny, nz, Y); break;
+        case 2: sh_all<2>(nx, ny, nz, Y); break;
+        default: sh_all<3>(nx, ny, nz, Y); break;
+      }
+      radial_basis<RM>(pl, rr, b);
+#pragma unroll
+      for (int m = 0; m < 16; ++m) geo[m] = Y[m].v;
+#pragma unroll
+      for (int k = 0; k < RM; ++k) geo[16 + k] = b[k].v;
+      if constexpr (DBL) {
+#pragma unroll
+        for (int m = 0; m < 16; ++m) geo[16 + RM + m] = Y[m].d[0];
+#pragma unroll
+        for (int k = 0; k < RM; ++k) geo[32 + RM + k] = b[k].d[0];
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < (DBL ? 32 : 16); ++m) acc[m] = 0.f;
+    float db[RM], hb[RM];
+#pragma unroll
+    for (int k = 0; k < RM; ++k) db[k] = hb[k] = 0.f;
+    for (int p = 0; p < pl.P; ++p) {
+      const DevPath& q = pl.path[p];
+      if (nb > 0) {
+        switch (triple_id(q.l1, q.l2, q.l3)) {
+#define TPC_CASE(a, b, c)                                                                                 \
+  case triple_id(a, b, c):                                                                                \
+    if constexpr (a <= LF && c <= LF)                                                                     \
+      wna_path<a, b, c, RM, DBL>(pl, q, L, ws, rl, nc, nb, myrow, x, x1, G, Gt, db, hb);                  \
+    break;
+          TPC_FOR_EACH_TRIPLE(TPC_CASE)
+#undef TPC_CASE
+          default: break;
+        }
+      }
+      __syncthreads();
+    }
+    if (valid) {
+      float v[3] = {vec[3 * e], vec[3 * e + 1], vec[3 * e + 2]};
+      float o3[3];
+      if constexpr (!DBL) {
+        if (dvec) {
+          edge_vec_grad<RM>(pl, v, acc, db, o3);
+          dvec[3 * e] = o3[0];
+          dvec[3 * e + 1] = o3[1];
+          dvec[3 * e + 2] = o3[2];
+        }
+        if (dYout)
+          for (int m = 0; m < pl.n_sh; ++m) dYout[size_t(e) * pl.n_sh + m] = acc[m];
+        if (dbout) {
+#pragma unroll
+          for (int k = 0; k < RM; ++k)
+            if (k < pl.R) dbout[size_t(e) * pl.R + k] = db[k];
+        }
+      } else {
+        float u[3] = {0.f, 0.f, 0.f};
+        if (ggv) load3(ggv, e, u);
+        edge_vec_grad2<RM>(pl, v, u, acc, acc + 16, db, hb, o3);
+        dvec[3 * e] = o3[0];
+        dvec[3 * e + 1] = o3[1];
+        dvec[3 * e + 2] = o3[2];
+      }
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace tpc

@@ -19,6 +19,7 @@
 #include <vector>
 
 #include "gemm_simt.cuh"
+#include "dtheta.h"
 #include "gemm_tc.h"
 #include "graph.cuh"
 #include "launchers.h"
@@ -54,9 +55,13 @@ int ensure_device() {
     if (tu.upload(t) != cudaSuccess) return TPCONV_ERR_CUDA;
     if (tu.smem && tu.smem(227 * 1024) != cudaSuccess) return TPCONV_ERR_CUDA;
   }
+  if (dtheta_smem_init() != cudaSuccess) return TPCONV_ERR_CUDA;
   g_ready[dev] = true;
   return TPCONV_OK;
 }
+
+// 16-byte aligned (or null): the adjoint streams stage feature rows with 16-byte copies
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 // ---- diagnostics: per-phase launch counts and optional event timing ----
 struct Profiler {
@@ -270,16 +275,7 @@ cudaError_t node_mix_sender(const tpconv_plan* plan, int s0, int nc, const float
       }
     }
   }
-  if (dtheta) {
-    for (int p = 0; p < d.P; ++p) {
-      const DevPath& q = d.path[p];
-      const int n1 = 2 * q.l1 + 1;
-      MView bp = mrow(F(B) + size_t(nc) * d.b_pref[q.i1] + q.kxoff, d.Kx[q.i1]);
-      MView xa = mview(F(x) + size_t(s0) * d.dim_in + q.in_off, 1, n1, 0, n1, d.dim_in, 1);
-      MView c = mview(dtheta + q.theta_off, 1, q.c_out, 0, q.c_out, int64_t(q.c_in) * q.c_out, 1);
-      if ((e = gemm_simt(q.c_in, int64_t(d.R) * q.c_out, int64_t(nc) * n1, xa, bp, c, 2, st))) return e;
-    }
-  }
+  if (dtheta && (e = dtheta_accumulate(d, s0, nc, x, B, nullptr, nullptr, dtheta, st))) return e;
   return cudaSuccess;
 }
 
@@ -394,8 +390,8 @@ int tpconv_forward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t*
     const int nc = int(std::min<int64_t>(L.chunk_nodes, N - r0));
     {
       PhaseScope ps(TPCONV_PHASE_FWD_EDGE, s);
-      if (TPC_RM_CALL(d.rm, launch_fwd_rm, d, int(r0), nc, rowptr, col, edge_vec, x, A, s)) return TPCONV_ERR_CUDA;
-      note(TPCONV_PHASE_FWD_EDGE, d.P);
+      if (TPC_WN_CALL_CPL(d, launch_wn_fwd, d, int(r0), nc, rowptr, col, edge_vec, x, A, s)) return TPCONV_ERR_CUDA;
+      note(TPCONV_PHASE_FWD_EDGE, 1);
     }
     {
       PhaseScope ps(TPCONV_PHASE_FWD_NODE, s);
@@ -446,9 +442,9 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
       }
       {
         PhaseScope ps(TPCONV_PHASE_BWD_EDGE_R, s);
-        cudaError_t e = d.pm_ok
-                            ? TPC_RM_CALL(d.rm, launch_adj_rm, d, int(r0), nc, rowptr, col, edge_vec, x, S_, dvec, dY,
-                                          db, s)
+        cudaError_t e = d.wn_ok && aligned16(x)
+                            ? TPC_WN_CALL(d, launch_wn_adj, d, int(r0), nc, rowptr, col, edge_vec, x, S_, dvec, dY, db,
+                                          s)
                             : TPC_RM_CALL(d.rm, launch_radj_rm, d, int(r0), nc, rowptr, col, edge_vec, x, S_, dvec,
                                           dY, db, s);
         if (e) return TPCONV_ERR_CUDA;
@@ -461,13 +457,13 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
       const int nc = int(std::min<int64_t>(L.chunk_nodes, N - s0));
       {
         PhaseScope ps(TPCONV_PHASE_BWD_EDGE_S, s);
-        if (TPC_RM_CALL(d.rm, launch_send_rm, d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, g, S_, s)) return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_BWD_EDGE_S, d.P);
+        if (TPC_WN_CALL_CPL(d, launch_wn_send, d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, g, S_, s)) return TPCONV_ERR_CUDA;
+        note(TPCONV_PHASE_BWD_EDGE_S, 1);
       }
       {
         PhaseScope ps(TPCONV_PHASE_BWD_NODE_X, s);
         if (node_mix_sender(plan, int(s0), nc, S_, x, theta, tcp, dx, dtheta, s)) return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_BWD_NODE_X, int64_t(dx ? d.n_in : 0) + int64_t(dtheta ? d.P : 0));
+        note(TPCONV_PHASE_BWD_NODE_X, int64_t(dx ? d.n_in : 0) + int64_t(dtheta ? 1 : 0));
       }
     }
   }
@@ -524,9 +520,9 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
       const int nc = int(std::min<int64_t>(Nc, N - r0));
       {
         PhaseScope ps(TPCONV_PHASE_DBL_EDGE_A, s);
-        if (TPC_RM_CALL(d.rm, launch_dbl_a_rm, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, A1, A0, s))
+        if (TPC_WN_CALL(d, launch_wn_dbla, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, A1, A0, s))
           return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_DBL_EDGE_A, d.P);
+        note(TPCONV_PHASE_DBL_EDGE_A, 1);
       }
       PhaseScope ps(TPCONV_PHASE_DBL_NODE_A, s);
       if (node_mix_forward(plan, int(r0), nc, A1, theta, t_hi, t_lo, d_g, s, 0)) return TPCONV_ERR_CUDA;
@@ -553,9 +549,9 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
         }
       }
       PhaseScope ps(TPCONV_PHASE_DBL_EDGE_R, s);
-      cudaError_t e = d.pm_ok
-                          ? TPC_RM_CALL(d.rm, launch_dadj_rm, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x,
-                                        gg_x, G, has_t ? Gt : nullptr, d_vec, s)
+      cudaError_t e = d.wn_ok && aligned16(x) && aligned16(gg_x)
+                          ? TPC_WN_CALL(d, launch_wn_dadj, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, G,
+                                        has_t ? Gt : nullptr, d_vec, s)
                           : TPC_RM_CALL(d.rm, launch_dbl_r_rm, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x,
                                         gg_x, G, has_t ? Gt : nullptr, d_vec, s);
       if (e) return TPCONV_ERR_CUDA;
@@ -570,20 +566,22 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
       const int nc = int(std::min<int64_t>(Nc, N - s0));
       {
         PhaseScope ps(TPCONV_PHASE_DBL_EDGE_S, s);
-        if (TPC_RM_CALL(d.rm, launch_dbl_s_rm, d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, gg_vec, g, B1, B0, s))
+        if (TPC_WN_CALL(d, launch_wn_dbls, d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, gg_vec, g, B1, B0, s))
           return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_DBL_EDGE_S, d.P);
+        note(TPCONV_PHASE_DBL_EDGE_S, 1);
       }
       PhaseScope ps(TPCONV_PHASE_DBL_NODE_X, s);
       float* dx1 = has_v ? d_x : nullptr;
       float* dt1 = has_v ? d_theta : nullptr;
-      if ((dx1 || dt1) && node_mix_sender(plan, int(s0), nc, B1, x, theta, tc0p, dx1, dt1, s)) return TPCONV_ERR_CUDA;
-      note(TPCONV_PHASE_DBL_NODE_X, int64_t(dx1 ? d.n_in : 0) + int64_t(dt1 ? d.P : 0));
+      if (dx1 && node_mix_sender(plan, int(s0), nc, B1, x, theta, tc0p, dx1, nullptr, s)) return TPCONV_ERR_CUDA;
       float* dx0 = has_t ? d_x : nullptr;
       float* dt0 = has_x1 ? d_theta : nullptr;
-      if ((dx0 || dt0) && node_mix_sender(plan, int(s0), nc, B0, gg_x, gg_theta, tc1p, dx0, dt0, s))
+      if (dx0 && node_mix_sender(plan, int(s0), nc, B0, gg_x, gg_theta, tc1p, dx0, nullptr, s)) return TPCONV_ERR_CUDA;
+      // d_theta = x^T B1 + gg_x^T B0 in one pass
+      if ((dt1 || dt0) && dtheta_accumulate(d, int(s0), nc, dt1 ? x : nullptr, dt1 ? B1 : nullptr, dt0 ? gg_x : nullptr,
+                                            dt0 ? B0 : nullptr, d_theta, s))
         return TPCONV_ERR_CUDA;
-      note(TPCONV_PHASE_DBL_NODE_X, int64_t(dx0 ? d.n_in : 0) + int64_t(dt0 ? d.P : 0));
+      note(TPCONV_PHASE_DBL_NODE_X, int64_t(dx1 ? d.n_in : 0) + int64_t(dx0 ? d.n_in : 0) + ((dt1 || dt0) ? 1 : 0));
     }
   }
   return finish(cudaSuccess);

@@ -1,0 +1,86 @@
+// Shared-memory layout of the warp-per-node edge streams (host and device).
+//
+// A warp owns one node: it walks the node's CSR segment and keeps every partial
+// sum of that node (lane = channel) or of its edges (lane = edge) in registers,
+// so the streams need no block-wide barrier and no cross-warp reduction.  Each
+// warp has its own slice of dynamic shared memory, laid out below in floats.
+#pragma once
+
+#if defined(__CUDACC__)
+#define TPC_HD __host__ __device__
+#else
+#define TPC_HD
+#endif
+
+namespace tpc {
+
+constexpr int kWnWarps = 4;   // warps (nodes) per CTA
+constexpr int kWnSub = 4;     // edges per staged sub-batch of the channel-lane streams
+constexpr int kWnChunk = 4;   // channels per staged chunk of the edge-lane (adjoint) streams
+
+// ---- lane = channel (receiver / sender forms, first and second order) ------
+// M, Md : coupling matrices of the 32 edges of the current geometry batch, nmp floats each
+// B, Bd : their radial bases, RM floats each
+// X, X1 : two sub-batch buffers of kWnSub staged neighbour rows, xs floats per row
+struct WnLay {
+  int M, Md, B, Bd, X, X1;
+  int nmp, xs, buf;  // buf = floats of one X buffer
+  int total;         // floats per warp
+};
+
+TPC_HD inline WnLay wn_layout_of(int RM, int cpl, int nimax, int nmz_max, bool dbl, bool two_src) {
+  WnLay L;
+  L.nmp = (nmz_max + 3) & ~3;
+  L.xs = (32 * cpl * nimax + 3) & ~3;
+  L.buf = kWnSub * L.xs;
+  L.M = 0;
+  L.Md = L.M + 32 * L.nmp;
+  L.B = L.Md + (dbl ? 32 * L.nmp : 0);
+  L.Bd = L.B + 32 * RM;
+  L.X = L.Bd + (dbl ? 32 * RM : 0);
+  L.X1 = L.X + 2 * L.buf;
+  L.total = L.X1 + (two_src ? 2 * L.buf : 0);
+  return L;
+}
+TPC_HD inline int wn_smem_bytes(int RM, int cpl, int nimax, int nmz_max, bool dbl, bool two_src) {
+  return kWnWarps * wn_layout_of(RM, cpl, nimax, nmz_max, dbl, two_src).total * 4;
+}
+
+// ---- lane = edge (receiver adjoint streams, first and second order) --------
+// G, Gt : two chunk buffers of kWnChunk channels of G (and Gt), [u][k][m3] with
+//         row stride RM * n3max (zero where never staged)
+// X, X1 : two chunk buffers of the 32 lanes' rows, [lane][u * n1 + m1] with row
+//         stride xs, xs / 4 odd: the 16-byte reads of 8 consecutive lanes fall
+//         into distinct bank quads
+// Geo   : per lane Y[16], b[RM] (and Yd[16], bd[RM]), odd stride
+// Acc   : per lane accumulators that persist across paths (dY, or wY and hY), odd stride
+struct WnaLay {
+  int G, Gt, X, X1, Geo, Acc;
+  int gs, gbuf, xs, xbuf, geos, accs;
+  int total;
+};
+
+TPC_HD inline WnaLay wna_layout_of(int RM, int n3max, int n1max, bool dbl) {
+  WnaLay L;
+  L.gs = RM * n3max;
+  L.gbuf = kWnChunk * L.gs;
+  L.xs = (kWnChunk * n1max + 3) & ~3;
+  if ((L.xs >> 2) % 2 == 0) L.xs += 4;
+  L.xbuf = 32 * L.xs;
+  L.geos = (dbl ? 2 : 1) * (16 + RM) + 1;
+  L.accs = (dbl ? 32 : 16) + 1;
+  L.G = 0;
+  L.Gt = L.G + 2 * L.gbuf;
+  L.X = L.Gt + (dbl ? 2 * L.gbuf : 0);
+  L.X1 = L.X + 2 * L.xbuf;
+  L.Geo = L.X1 + (dbl ? 2 * L.xbuf : 0);
+  L.Acc = L.Geo + 32 * L.geos;
+  L.total = (L.Acc + 32 * L.accs + 3) & ~3;
+  return L;
+}
+// the warps' slices and one int (the CTA's batch count)
+TPC_HD inline int wna_smem_bytes(int RM, int n3max, int n1max, bool dbl) {
+  return kWnWarps * wna_layout_of(RM, n3max, n1max, dbl).total * 4 + 16;
+}
+
+}  // namespace tpc
