@@ -19,6 +19,7 @@ sample of the same workload (the pages ship no runnable reference).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import subprocess
@@ -68,6 +69,18 @@ def measured_peaks():
 # ---------------------------------------------------------------------------
 # algorithmic work model (per edge), from the plan's path table and CG pattern
 # ---------------------------------------------------------------------------
+def sources_digest():
+    """Digest of the CUDA/C++ sources: DRAM counters taken on other sources do not apply."""
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "equivariant_gnn_tensor_receiver_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
+            h.update(f.encode())
+            with open(os.path.join(d, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()
+
+
 def work_model(T, plan):
     R = plan.R
     nnz_cache = {}
@@ -82,10 +95,10 @@ def work_model(T, plan):
         n1, n3 = 2 * p["l1"] + 1, 2 * p["l3"] + 1
         ci, co = p["c_in"], p["c_out"]
         fw += nnz + ci * (mnz + R * n3)                           # M_e, M x, b (x) T
-        bw_r += nnz + ci * (mnz + 2 * R * n3 + mnz + nnz)         # M x, dT, db, C(x, dT)
+        bw_r += 2 * nnz + ci * (2 * mnz + 2 * R * n3)             # M_e; M x, dT, db, Q += x (x) dT; C : Q
         bw_s += nnz + co * (mnz + R * n1)                         # M_e, M^T g, b (x) U
         db_a += 2 * nnz + ci * (3 * mnz + 3 * R * n3)
-        db_r += 2 * nnz + ci * (3 * mnz + 6 * R * n3 + 3 * (mnz + nnz))
+        db_r += 4 * nnz + ci * (6 * mnz + 6 * R * n3)             # M, Md; 3 M-products, 3 Q updates; C : Qw, Qh
         db_s += 2 * nnz + co * (2 * mnz + 3 * R * n1)
     return {"fwd_edge": fw, "bwd_edge_r": bw_r, "bwd_edge_s": bw_s, "dbl_edge_a": db_a, "dbl_edge_r": db_r,
             "dbl_edge_s": db_s}
@@ -347,8 +360,9 @@ def run_ours(args):
     try:
         with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
             tr = json.load(f).get(dom)
-        if tr and tr.get("lib_mtime") == int(os.path.getmtime(L.LIB_PATH)):
-            roof["traffic"] = tr["bytes_per_step"]
+        if tr and tr.get("sources_sha256") == sources_digest():
+            roof["traffic"] = tr["dram_bytes_per_launch"]
+            roof["traffic_kernel"] = tr["kernel"]
     except (OSError, ValueError):
         pass
 
