@@ -17,6 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtpconv.so")
 
 TPCONV_OK = 0
+TPCONV_ERR_WORKSPACE_TOO_SMALL = 4
 STATUS = {0: "ok", 1: "invalid argument", 2: "bad irreps", 3: "unsupported", 4: "workspace too small",
           5: "CUDA error", 6: "graph invalid", 7: "timeout", 8: "internal"}
 RADIAL = {"gaussian": 0, "bessel": 1}
@@ -54,6 +55,7 @@ _EXPORTS = {
     "tpconv_workspace_size": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, ctypes.POINTER(ctypes.c_size_t)]),
     "tpconv_graph_transpose": (ctypes.c_int, [_P, _I64, _I64] + [_P] * 5 + [_P, ctypes.c_size_t, _P]),
     "tpconv_forward": (ctypes.c_int, [_P, _I64, _I64] + [_P] * 6 + [_P, ctypes.c_size_t, _P]),
+    "tpconv_forward_static": (ctypes.c_int, [_P, _I64, _I64] + [_P] * 6 + [_P]),
     "tpconv_backward": (ctypes.c_int, [_P, _I64, _I64] + [_P] * 14 + [_P, ctypes.c_size_t, _P]),
     "tpconv_double_backward": (ctypes.c_int, [_P, _I64, _I64] + [_P] * 16 + [_P, ctypes.c_size_t, _P]),
     "tpconv_profile_enable": (ctypes.c_int, [ctypes.c_int]),
@@ -199,6 +201,14 @@ def tpconv_forward(plan, N, E, rowptr, col, edge_vec, x, theta, out, workspace, 
     _check("tpconv_forward",
            lib().tpconv_forward(plan.handle, N, E, _ptr(rowptr, i32), _ptr(col, i32), _ptr(edge_vec, f32),
                                 _ptr(x, f32), _ptr(theta, f32), _ptr(out, f32), w, wb, _stream(stream)))
+
+
+def tpconv_forward_static(plan, N, E, rowptr, col, edge_vec, x, theta, out, stream=None):
+    import torch
+    f32, i32 = torch.float32, torch.int32
+    _check("tpconv_forward_static",
+           lib().tpconv_forward_static(plan.handle, N, E, _ptr(rowptr, i32), _ptr(col, i32), _ptr(edge_vec, f32),
+                                       _ptr(x, f32), _ptr(theta, f32), _ptr(out, f32), _stream(stream)))
 
 
 def tpconv_backward(plan, N, E, rowptr, col, perm, s_rowptr, s_recv, edge_vec, x, theta, g, dx, dtheta, dvec,

@@ -158,6 +158,32 @@ int tpconv_forward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t*
                    float* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Allocation-free forward (device, async).  No counterpart in the pages: an
+ * interface addition of this library for callers that cannot allocate device
+ * memory (a host program without a device allocator of its own, a plugin that
+ * may not bypass its framework's caching allocator, a fixed-latency loop that
+ * must not call cudaMalloc, which can synchronise the device).
+ *
+ * Same arguments and result as tpconv_forward, without workspace: the
+ * workspace is a fixed array of TPCONV_STATIC_SCRATCH_BYTES inside the library
+ * (one per device).  Nothing is allocated.  Nothing in it needs to start at
+ * zero.
+ *   Returns TPCONV_ERR_WORKSPACE_TOO_SMALL, before any device work, when
+ *   tpconv_workspace_size(plan, TPCONV_OP_FORWARD, N, E) exceeds
+ *   TPCONV_STATIC_SCRATCH_BYTES; a plan created with a smaller workspace_cap
+ *   (node chunks) fits.
+ *   Calls share the array: calls that overlap in time (other streams, other
+ *   host threads) race on it and must be serialised by the caller.
+ *   The first call on a device also performs the library's one-time device
+ *   set-up (constant tables, kernel attributes, the array's address), which
+ *   synchronises the device: make it before any stream capture.
+ */
+#define TPCONV_STATIC_SCRATCH_BYTES (64u << 20) /* 64 MiB */
+int tpconv_forward_static(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t* rowptr,
+                          const int32_t* col, const float* edge_vec, const float* x, const float* theta,
+                          float* out, void* stream);
+
+/*
  * Backward (device, async) for the cotangent g[N][dim_out] of out.
  *   dx[N][dim_in], dtheta[theta_numel], dvec[E][3] (CSR order): optional.
  *   dY[E][n_sh], db[E][R]: optional per-edge adjoints of the spherical
