@@ -69,15 +69,14 @@ def measured_peaks():
 # ---------------------------------------------------------------------------
 # algorithmic work model (per edge), from the plan's path table and CG pattern
 # ---------------------------------------------------------------------------
-def sources_digest():
-    """Digest of the CUDA/C++ sources: DRAM counters taken on other sources do not apply."""
+def sources_digest(files):
+    """Digest of the named CUDA/C++ sources of a kernel: counters taken on other sources do not apply."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "equivariant_gnn_tensor_receiver_b200", "csrc")
-    for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
-            h.update(f.encode())
-            with open(os.path.join(d, f), "rb") as fh:
-                h.update(fh.read())
+    for f in sorted(files):
+        h.update(f.encode())
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()
 
 
@@ -360,7 +359,7 @@ def run_ours(args):
     try:
         with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
             tr = json.load(f).get(dom)
-        if tr and tr.get("sources_sha256") == sources_digest():
+        if tr and tr.get("sources_sha256") == sources_digest(tr["sources"]):
             roof["traffic"] = tr["dram_bytes_per_launch"]
             roof["traffic_kernel"] = tr["kernel"]
     except (OSError, ValueError):
