@@ -41,6 +41,17 @@ __device__ __forceinline__ void lds_vec(const float* p, float* v) {
     v[4 * i + 3] = t.w;
   }
 }
+// load NP (even) consecutive float pairs from 16-byte aligned shared memory
+template <int NP>
+__device__ __forceinline__ void lds_f2(const float* p, float2* v) {
+  static_assert(NP % 2 == 0, "pairs come in 16-byte groups");
+#pragma unroll
+  for (int i = 0; i < NP / 2; ++i) {
+    const float4 t = lds4(p + 4 * i);
+    v[2 * i] = make_float2(t.x, t.y);
+    v[2 * i + 1] = make_float2(t.z, t.w);
+  }
+}
 template <int N>
 __device__ __forceinline__ void sts_vec(float* p, const float* v) {
   static_assert(N % 4 == 0, "vector width");

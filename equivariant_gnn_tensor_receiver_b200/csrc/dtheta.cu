@@ -10,7 +10,7 @@
 // 64 (u) x 256 (k, w) tile; stages of about 40 K rows are gathered with cp.async
 // into a double buffer (x transposed to [row][u] on the way in), and each
 // thread keeps an 8 x 8 accumulator tile fed by four 16-byte shared reads per
-// 64 FFMA (the u quad is a warp-wide broadcast).
+// 32 paired FMAs (the u octet is a warp-wide broadcast).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -96,11 +96,11 @@ __device__ __forceinline__ void tile(const DevPlan& pl, const DevPath& q, int u0
     dt_stage<N1>(sm + (it & 1) * kStageMax, ns, x, size_t(s0 + sc) * pl.dim_in + q.in_off + size_t(u0) * N1,
                  pl.dim_in, cu, B, size_t(sc) * N1 * ldb, ldb, cn, v4);
   };
-  float acc[8][8];
+  float2 acc[8][4];  // column pairs (2cp, 2cp+1) of the thread's 8 columns
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
+    for (int c = 0; c < 4; ++c) acc[i][c] = make_float2(0.f, 0.f);
   if (nst > 0) stage(0);
   ac_commit();
   for (int it = 0; it < nst; ++it) {
@@ -113,16 +113,17 @@ __device__ __forceinline__ void tile(const DevPlan& pl, const DevPath& q, int u0
     const int sc = sb + (it % nst1) * C::TS;
     const int rows = min(C::TS, se - sc) * N1;
     for (int r = 0; r < rows; ++r) {
-      float a[8], b[8];
+      float a[8];
+      float2 b[4];
       lds_vec<8>(sX + r * kTU + 8 * warp, a);
-      const float4 b0 = lds4(sB + r * kTN + 4 * lane);
-      const float4 b1 = lds4(sB + r * kTN + 128 + 4 * lane);
-      b[0] = b0.x; b[1] = b0.y; b[2] = b0.z; b[3] = b0.w;
-      b[4] = b1.x; b[5] = b1.y; b[6] = b1.z; b[7] = b1.w;
+      lds_f2<2>(sB + r * kTN + 4 * lane, b);
+      lds_f2<2>(sB + r * kTN + 128 + 4 * lane, b + 2);
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int i = 0; i < 8; ++i) {
+        const float2 ai = make_float2(a[i], a[i]);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[i][c] = fmaf(a[i], b[c], acc[i][c]);
+        for (int c = 0; c < 4; ++c) acc[i][c] = __ffma2_rn(ai, b[c], acc[i][c]);
+      }
     }
     __syncthreads();
   }
@@ -136,7 +137,8 @@ __device__ __forceinline__ void tile(const DevPlan& pl, const DevPath& q, int u0
       const int n = c < 4 ? 4 * lane + c : 128 + 4 * lane + c - 4;
       if (n >= cn) continue;
       const int ng = n0 + n, k = ng / q.c_out, w = ng - k * q.c_out;
-      atomicAdd(dtheta + q.theta_off + (size_t(k) * q.c_in + u0 + u) * q.c_out + w, acc[i][c]);
+      const float v = (c & 1) ? acc[i][c >> 1].y : acc[i][c >> 1].x;
+      atomicAdd(dtheta + q.theta_off + (size_t(k) * q.c_in + u0 + u) * q.c_out + w, v);
     }
   }
 }

@@ -76,7 +76,12 @@ __device__ __forceinline__ void wn_coupling(const float* Y, float* Mrow) {
   for (int i = NMZ; i < NMP; ++i) Mrow[i] = 0.f;
 }
 
-// one path, all channel tiles of the warp's node
+// (a.x, a.y) = (b.x, b.y) * (t, t) + (a.x, a.y): two FP32 FMAs in one instruction
+__device__ __forceinline__ void ffma2_bcast(float2& a, float2 b, float t) { a = __ffma2_rn(b, make_float2(t, t), a); }
+
+// one path, all channel tiles of the warp's node.  The radial state is kept as
+// float2 pairs of consecutive radial indices, so the outer products b (x) T run
+// as paired FMAs; shared-memory strides are the path's own compile-time widths.
 template <int L1, int L2, int L3, int RM, int CPL, bool RECV, bool DBL>
 __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q, const WnLay& L, float* ws, int nl,
                                              int nc, int a0, int a1, const int* __restrict__ nbr,
@@ -89,7 +94,10 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
   constexpr int NI = RECV ? TR::N1 : TR::N3;  // staged floats per channel
   constexpr int NO = RECV ? TR::N3 : TR::N1;  // state floats per channel and radial index
   constexpr int NPART = DBL ? 2 : 1;
-  constexpr int NACC = NPART * CPL * RM * NO;
+  constexpr int NK2 = RM / 2;                 // radial pairs
+  constexpr int NACC = NPART * CPL * NK2 * NO;
+  constexpr int XS = (32 * CPL * NI + 3) & ~3;  // staged row stride of this path (<= L.xs)
+  constexpr int BUF = kWnSub * XS;
   const int lane = lane_id();
   const int c = RECV ? q.c_in : q.c_out;
   const int dim = RECV ? pl.dim_in : pl.dim_out;
@@ -101,37 +109,43 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
   float* sMd = ws + L.Md;
   float* sB = ws + L.B;
   float* sBd = ws + L.Bd;
+  float* sX = ws + L.X;
+  float* sX1 = ws + L.X1;
 
   for (int c0 = 0; c0 < c; c0 += 32 * CPL) {
     const int w = min(32 * CPL, c - c0);
     const int len = w * NI;
     const bool v4 = ((dim | off | len) & 3) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0 &&
                     (reinterpret_cast<uintptr_t>(src1) & 15) == 0;
-    const size_t coff = size_t(off) + size_t(c0) * NI;
+    const float* srcc = src + size_t(off) + size_t(c0) * NI;
+    const float* src1c = two ? src1 + size_t(off) + size_t(c0) * NI : nullptr;
     // stage the rows of sub-batch sb into buffer sb & 1 (one commit group per call site)
     auto stage = [&](int sb) {
       const int j0 = sb * kWnSub, nb = min(kWnSub, ne - j0);
-      float* X = ws + L.X + (sb & 1) * L.buf;
-      float* X1 = ws + L.X1 + (sb & 1) * L.buf;
+      float* X = sX + (sb & 1) * BUF;
+      float* X1 = sX1 + (sb & 1) * BUF;
+      const int* nb_idx = nbr + a0 + j0;
       for (int j = 0; j < nb; ++j) {
-        const size_t row = size_t(nbr[a0 + j0 + j]) * dim + coff;
+        const size_t row = size_t(nb_idx[j]) * dim;
+        const float* rs = srcc + row;
+        float* xd = X + j * XS;
         if (v4) {
           for (int o = 4 * lane; o < len; o += 128) {
-            ac_copy16(X + j * L.xs + o, src + row + o);
-            if (two) ac_copy16(X1 + j * L.xs + o, src1 + row + o);
+            ac_copy16(xd + o, rs + o);
+            if (two) ac_copy16(X1 + j * XS + o, src1c + row + o);
           }
         } else {
           for (int o = lane; o < len; o += 32) {
-            ac_copy4(X + j * L.xs + o, src + row + o);
-            if (two) ac_copy4(X1 + j * L.xs + o, src1 + row + o);
+            ac_copy4(xd + o, rs + o);
+            if (two) ac_copy4(X1 + j * XS + o, src1c + row + o);
           }
         }
       }
     };
 
-    float acc[NACC];
+    float2 acc[NACC];
 #pragma unroll
-    for (int i = 0; i < NACC; ++i) acc[i] = 0.f;
+    for (int i = 0; i < NACC; ++i) acc[i] = make_float2(0.f, 0.f);
 
     if (nsb > 0) stage(0);
     ac_commit();
@@ -146,11 +160,11 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
           float Y[N2], Yd[N2], b[RM], bd[RM], Mrow[NMP];
           wn_geometry<L2, RM, DBL>(pl, vec, ggv, e, Y, Yd, b, bd);
           wn_coupling<L1, L2, L3, NMP>(Y, Mrow);
-          sts_vec<NMP>(sM + lane * L.nmp, Mrow);
+          sts_vec<NMP>(sM + lane * NMP, Mrow);
           sts_vec<RM>(sB + lane * RM, b);
           if constexpr (DBL) {
             wn_coupling<L1, L2, L3, NMP>(Yd, Mrow);
-            sts_vec<NMP>(sMd + lane * L.nmp, Mrow);
+            sts_vec<NMP>(sMd + lane * NMP, Mrow);
             sts_vec<RM>(sBd + lane * RM, bd);
           }
         }
@@ -160,61 +174,67 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
       ac_commit();
       ac_wait<1>();
       __syncwarp();
-      const float* X = ws + L.X + (sb & 1) * L.buf;
-      const float* X1 = ws + L.X1 + (sb & 1) * L.buf;
       const int nb = min(kWnSub, ne - j0);
-      for (int jj = 0; jj < nb; ++jj) {
-        const int js = (j0 & 31) + jj;
-        float Mv[NMP], bv[RM];
-        lds_vec<NMP>(sM + js * L.nmp, Mv);
-        lds_vec<RM>(sB + js * RM, bv);
-        float Mdv[DBL ? NMP : 1], bdv[DBL ? RM : 1];
+      const float* Mp = sM + (j0 & 31) * NMP;
+      const float* Mdp = sMd + (j0 & 31) * NMP;
+      const float* Bp = sB + (j0 & 31) * RM;
+      const float* Bdp = sBd + (j0 & 31) * RM;
+      const float* Xp = sX + (sb & 1) * BUF + lane * NI;
+      const float* X1p = sX1 + (sb & 1) * BUF + lane * NI;
+      for (int jj = 0; jj < nb; ++jj, Mp += NMP, Mdp += NMP, Bp += RM, Bdp += RM, Xp += XS, X1p += XS) {
+        float Mv[NMP];
+        float2 b2[NK2];
+        lds_vec<NMP>(Mp, Mv);
+        lds_f2<NK2>(Bp, b2);
+        float Mdv[DBL ? NMP : 1];
+        float2 bd2[DBL ? NK2 : 1];
         if constexpr (DBL) {
-          lds_vec<NMP>(sMd + js * L.nmp, Mdv);
-          lds_vec<RM>(sBd + js * RM, bdv);
+          lds_vec<NMP>(Mdp, Mdv);
+          lds_f2<NK2>(Bdp, bd2);
         }
 #pragma unroll
         for (int h = 0; h < CPL; ++h) {
-          const int cb = jj * L.xs + (lane + 32 * h) * NI;
           float xv[NI];
 #pragma unroll
-          for (int i = 0; i < NI; ++i) xv[i] = X[cb + i];
-          float* a = acc + h * RM * NO;                  // part 0
-          float* a1 = acc + (CPL + h) * RM * NO;         // part 1 (second order)
+          for (int i = 0; i < NI; ++i) xv[i] = Xp[32 * NI * h + i];
+          float2* a = acc + h * NK2 * NO;                 // part 0
+          float2* a1 = acc + (CPL + h) * NK2 * NO;        // part 1 (second order)
           if constexpr (!DBL) {
             float T[NO];
             if constexpr (RECV) apply_M<L1, L2, L3>(Mv, xv, T);
             else apply_Mt<L1, L2, L3>(Mv, xv, T);
 #pragma unroll
-            for (int k = 0; k < RM; ++k)
+            for (int kp = 0; kp < NK2; ++kp)
 #pragma unroll
-              for (int i = 0; i < NO; ++i) a[k * NO + i] = fmaf(bv[k], T[i], a[k * NO + i]);
+              for (int i = 0; i < NO; ++i) ffma2_bcast(a[kp * NO + i], b2[kp], T[i]);
           } else if constexpr (RECV) {
             float x1v[NI], T[NO], T1[NO], T2[NO];
 #pragma unroll
-            for (int i = 0; i < NI; ++i) x1v[i] = two ? X1[cb + i] : 0.f;
+            for (int i = 0; i < NI; ++i) x1v[i] = two ? X1p[i] : 0.f;
             apply_M<L1, L2, L3>(Mv, xv, T);
             apply_M<L1, L2, L3>(Mv, x1v, T1);
             apply_M<L1, L2, L3>(Mdv, xv, T2);
 #pragma unroll
             for (int i = 0; i < NO; ++i) T1[i] += T2[i];
 #pragma unroll
-            for (int k = 0; k < RM; ++k)
+            for (int kp = 0; kp < NK2; ++kp)
 #pragma unroll
               for (int i = 0; i < NO; ++i) {
-                a[k * NO + i] = fmaf(bv[k], T1[i], fmaf(bdv[k], T[i], a[k * NO + i]));
-                a1[k * NO + i] = fmaf(bv[k], T[i], a1[k * NO + i]);
+                ffma2_bcast(a[kp * NO + i], bd2[kp], T[i]);
+                ffma2_bcast(a[kp * NO + i], b2[kp], T1[i]);
+                ffma2_bcast(a1[kp * NO + i], b2[kp], T[i]);
               }
           } else {
             float U[NO], U1[NO];
             apply_Mt<L1, L2, L3>(Mv, xv, U);
             apply_Mt<L1, L2, L3>(Mdv, xv, U1);
 #pragma unroll
-            for (int k = 0; k < RM; ++k)
+            for (int kp = 0; kp < NK2; ++kp)
 #pragma unroll
               for (int i = 0; i < NO; ++i) {
-                a[k * NO + i] = fmaf(bv[k], U1[i], fmaf(bdv[k], U[i], a[k * NO + i]));
-                a1[k * NO + i] = fmaf(bv[k], U[i], a1[k * NO + i]);
+                ffma2_bcast(a[kp * NO + i], bd2[kp], U[i]);
+                ffma2_bcast(a[kp * NO + i], b2[kp], U1[i]);
+                ffma2_bcast(a1[kp * NO + i], b2[kp], U[i]);
               }
           }
         }
@@ -234,12 +254,14 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
         const int ch = lane + 32 * h;
         if (ch >= w) continue;
 #pragma unroll
-        for (int k = 0; k < RM; ++k) {
-          if (k >= pl.R) break;
+        for (int kp = 0; kp < NK2; ++kp)
 #pragma unroll
-          for (int i = 0; i < NO; ++i)
-            dst[base + size_t(i) * Kq + k * c + ch] = acc[((part * CPL + h) * RM + k) * NO + i];
-        }
+          for (int i = 0; i < NO; ++i) {
+            const float2 v = acc[((part * CPL + h) * NK2 + kp) * NO + i];
+            float* d = dst + base + size_t(i) * Kq + ch;
+            if (2 * kp < pl.R) d[size_t(2 * kp) * c] = v.x;
+            if (2 * kp + 1 < pl.R) d[size_t(2 * kp + 1) * c] = v.y;
+          }
       }
     }
   }

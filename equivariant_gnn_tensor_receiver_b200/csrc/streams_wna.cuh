@@ -60,35 +60,45 @@ __device__ __forceinline__ void contract_Q(const float* Q, float* out) {
   });
 }
 
+// Shared G tiles hold radial pairs side by side, [u][k / 2][m3][k & 1], so that a
+// 16-byte read yields float2 operands (G_2kp, G_2kp+1) for paired FMAs.
+template <int N3>
+__host__ __device__ constexpr int g_slot(int k, int m3) {
+  return ((k >> 1) * N3 + m3) * 2 + (k & 1);
+}
+
 // one path of one 32-edge batch
 template <int L1, int L2, int L3, int RM, bool DBL>
 __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, const WnaLay& L, float* ws, int rl,
                                          int nc, int nb, int myrow, const float* __restrict__ x,
                                          const float* __restrict__ x1, const float* __restrict__ G,
-                                         const float* __restrict__ Gt, float* db, float* hb) {
+                                         const float* __restrict__ Gt, float2* db, float2* hb) {
   using TR = Tri<L1, L2, L3>;
-  constexpr int N1 = TR::N1, N2 = TR::N2, N3 = TR::N3, NMZ = TR::NMZ, GW = RM * N3;
+  constexpr int N1 = TR::N1, N2 = TR::N2, N3 = TR::N3, NMZ = TR::NMZ, GW = RM * N3, NK2 = RM / 2;
   constexpr int CH = kWnChunk;
   static_assert(CH == 4, "the chunk is one group of four channels");
+  constexpr int NIT = (GW * CH + 31) / 32;  // G elements per lane and chunk (upper bound)
   const int lane = lane_id();
   const float* geo = ws + L.Geo + lane * L.geos;
-  float Mv[NMZ], bv[RM];
+  float Mv[NMZ];
+  float2 b2[NK2];
   {
     float Y[N2];
 #pragma unroll
     for (int i = 0; i < N2; ++i) Y[i] = geo[L2 * L2 + i];
     coupling_row<L1, L2, L3>(Y, Mv);
 #pragma unroll
-    for (int k = 0; k < RM; ++k) bv[k] = geo[16 + k];
+    for (int kp = 0; kp < NK2; ++kp) b2[kp] = make_float2(geo[16 + 2 * kp], geo[17 + 2 * kp]);
   }
-  float Mdv[DBL ? NMZ : 1], bdv[DBL ? RM : 1];
+  float Mdv[DBL ? NMZ : 1];
+  float2 bd2[DBL ? NK2 : 1];
   if constexpr (DBL) {
     float Y[N2];
 #pragma unroll
     for (int i = 0; i < N2; ++i) Y[i] = geo[16 + RM + L2 * L2 + i];
     coupling_row<L1, L2, L3>(Y, Mdv);
 #pragma unroll
-    for (int k = 0; k < RM; ++k) bdv[k] = geo[32 + RM + k];
+    for (int kp = 0; kp < NK2; ++kp) bd2[kp] = make_float2(geo[32 + RM + 2 * kp], geo[33 + RM + 2 * kp]);
   }
   float Q[NMZ], Qh[DBL ? NMZ : 1];
 #pragma unroll
@@ -101,18 +111,30 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
   const int c = q.c_in, R = pl.R;
   const int nch = c / CH;  // channel counts are multiples of four on this path
   const int Kb = pl.Kb[q.i3];
-  const size_t gbase = size_t(nc) * pl.a_pref[q.i3] + size_t(rl) * N3 * Kb + q.koff;
   const bool has_t = DBL && Gt != nullptr, has_x1 = DBL && x1 != nullptr;
+  // this lane's G elements of a chunk: source offset (relative to channel u0)
+  // and shared slot, the same for every chunk of the path
+  const float* Gp = G + size_t(nc) * pl.a_pref[q.i3] + size_t(rl) * N3 * Kb + q.koff;
+  const float* Gtp = has_t ? Gt + (Gp - G) : nullptr;
+  int gsrc[NIT], gdst[NIT];
+#pragma unroll
+  for (int it = 0; it < NIT; ++it) {
+    const int t = it * 32 + lane;
+    const int u = t & (CH - 1), km = t / CH;  // km = k * N3 + m3
+    const int k = km / N3, m3 = km - k * N3;
+    gsrc[it] = k < R ? m3 * Kb + k * c + u : -1;
+    gdst[it] = u * GW + g_slot<N3>(k, m3);
+  }
   auto stage = [&](int ch) {
     const int u0 = ch * CH;
     float* sG = ws + L.G + (ch & 1) * L.gbuf;
     float* sGt = ws + L.Gt + (ch & 1) * L.gbuf;
-    for (int t = lane; t < R * N3 * CH; t += 32) {
-      const int u = t & (CH - 1), km = t / CH;  // km = k * N3 + m3
-      const int k = km / N3, m3 = km - k * N3;
-      const size_t src = gbase + size_t(m3) * Kb + size_t(k) * c + u0 + u;
-      ac_copy4(sG + u * L.gs + km, G + src);
-      if (has_t) ac_copy4(sGt + u * L.gs + km, Gt + src);
+#pragma unroll
+    for (int it = 0; it < NIT; ++it) {
+      if (gsrc[it] >= 0) {
+        ac_copy4(sG + gdst[it], Gp + u0 + gsrc[it]);
+        if (has_t) ac_copy4(sGt + gdst[it], Gtp + u0 + gsrc[it]);
+      }
     }
     // the batch's rows, N1 16-byte pieces each, copied by the whole warp (coalesced)
     float* sX = ws + L.X + (ch & 1) * L.xbuf;
@@ -147,57 +169,63 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
 #pragma unroll
     for (int t = 0; t < CH; ++t) {
       const float* xv = xg + t * N1;
-      const float* x1v = DBL ? x1g + t * N1 : xv;
       float T[N3];
       apply_M<L1, L2, L3>(Mv, xv, T);
       if constexpr (!DBL) {
-        float g[GW];
-        lds_vec<GW>(sG + t * L.gs, g);
-        float dT[N3];
+        float2 g2[NK2 * N3];
+        lds_f2<NK2 * N3>(sG + t * GW, g2);
+        float2 dT2[N3];
 #pragma unroll
-        for (int i = 0; i < N3; ++i) dT[i] = 0.f;
+        for (int i = 0; i < N3; ++i) dT2[i] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int k = 0; k < RM; ++k) {
-          float s = 0.f;
+        for (int kp = 0; kp < NK2; ++kp)
 #pragma unroll
           for (int i = 0; i < N3; ++i) {
-            dT[i] = fmaf(bv[k], g[k * N3 + i], dT[i]);
-            s = fmaf(g[k * N3 + i], T[i], s);
+            const float2 g = g2[kp * N3 + i];
+            dT2[i] = __ffma2_rn(b2[kp], g, dT2[i]);
+            db[kp] = __ffma2_rn(g, make_float2(T[i], T[i]), db[kp]);
           }
-          db[k] += s;
-        }
+        float dT[N3];
+#pragma unroll
+        for (int i = 0; i < N3; ++i) dT[i] = dT2[i].x + dT2[i].y;
         outer_Q<L1, L2, L3>(xv, dT, Q);
       } else {
+        const float* x1v = x1g + t * N1;
         float T12[N3], Tb[N3];
         apply_M<L1, L2, L3>(Mv, x1v, T12);
         apply_M<L1, L2, L3>(Mdv, xv, Tb);
 #pragma unroll
         for (int i = 0; i < N3; ++i) T12[i] += Tb[i];
-        float dG[N3], dX[N3];
+        float2 dG2[N3], dX2[N3];
 #pragma unroll
-        for (int i = 0; i < N3; ++i) dG[i] = dX[i] = 0.f;
-        // G and Gt rows in KH slices of RM / KH radial indices (bounds the live registers)
-        constexpr int KH = RM >= 8 ? 2 : 1, KS = RM / KH;
+        for (int i = 0; i < N3; ++i) dG2[i] = dX2[i] = make_float2(0.f, 0.f);
+        // G and Gt rows in KH slices of radial pairs (bounds the live registers)
+        constexpr int KH = NK2 >= 4 ? 2 : 1, KS = NK2 / KH;  // KS pairs per slice
 #pragma unroll
         for (int kh = 0; kh < KH; ++kh) {
-          float g[KS * N3], gt[KS * N3];
-          lds_vec<KS * N3>(sG + t * L.gs + kh * KS * N3, g);
-          lds_vec<KS * N3>(sGt + t * L.gs + kh * KS * N3, gt);
+          float2 g2[KS * N3], gt2[KS * N3];
+          lds_f2<KS * N3>(sG + t * GW + 2 * kh * KS * N3, g2);
+          lds_f2<KS * N3>(sGt + t * GW + 2 * kh * KS * N3, gt2);
 #pragma unroll
           for (int kk = 0; kk < KS; ++kk) {
-            const int k = kh * KS + kk;
-            float s1 = 0.f, s0 = 0.f;
+            const int kp = kh * KS + kk;
 #pragma unroll
             for (int i = 0; i < N3; ++i) {
-              const float gv = g[kk * N3 + i], tv = gt[kk * N3 + i];
-              dG[i] = fmaf(bv[k], gv, dG[i]);
-              dX[i] = fmaf(bv[k], tv, fmaf(bdv[k], gv, dX[i]));
-              s1 = fmaf(gv, T12[i], fmaf(tv, T[i], s1));
-              s0 = fmaf(gv, T[i], s0);
+              const float2 g = g2[kk * N3 + i], gt = gt2[kk * N3 + i];
+              dG2[i] = __ffma2_rn(b2[kp], g, dG2[i]);
+              dX2[i] = __ffma2_rn(bd2[kp], g, dX2[i]);
+              dX2[i] = __ffma2_rn(b2[kp], gt, dX2[i]);
+              db[kp] = __ffma2_rn(gt, make_float2(T[i], T[i]), db[kp]);
+              db[kp] = __ffma2_rn(g, make_float2(T12[i], T12[i]), db[kp]);
+              hb[kp] = __ffma2_rn(g, make_float2(T[i], T[i]), hb[kp]);
             }
-            db[k] += s1;
-            hb[k] += s0;
           }
+        }
+        float dG[N3], dX[N3];
+#pragma unroll
+        for (int i = 0; i < N3; ++i) {
+          dG[i] = dG2[i].x + dG2[i].y;
+          dX[i] = dX2[i].x + dX2[i].y;
         }
         outer_Q<L1, L2, L3>(x1v, dG, Q);
         outer_Q<L1, L2, L3>(xv, dX, Q);
@@ -294,9 +322,9 @@ __global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
     }
 #pragma unroll
     for (int m = 0; m < (DBL ? 32 : 16); ++m) acc[m] = 0.f;
-    float db[RM], hb[RM];
+    float2 db2[RM / 2], hb2[RM / 2];  // radial pairs (2kp, 2kp+1)
 #pragma unroll
-    for (int k = 0; k < RM; ++k) db[k] = hb[k] = 0.f;
+    for (int kp = 0; kp < RM / 2; ++kp) db2[kp] = hb2[kp] = make_float2(0.f, 0.f);
     for (int p = 0; p < pl.P; ++p) {
       const DevPath& q = pl.path[p];
       if (nb > 0) {
@@ -304,7 +332,7 @@ __global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
 #define TPC_CASE(a, b, c)                                                                                 \
   case triple_id(a, b, c):                                                                                \
     if constexpr (a <= LF && c <= LF)                                                                     \
-      wna_path<a, b, c, RM, DBL>(pl, q, L, ws, rl, nc, nb, myrow, x, x1, G, Gt, db, hb);                  \
+      wna_path<a, b, c, RM, DBL>(pl, q, L, ws, rl, nc, nb, myrow, x, x1, G, Gt, db2, hb2);                  \
     break;
           TPC_FOR_EACH_TRIPLE(TPC_CASE)
 #undef TPC_CASE
@@ -315,7 +343,14 @@ __global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
     }
     if (valid) {
       float v[3] = {vec[3 * e], vec[3 * e + 1], vec[3 * e + 2]};
-      float o3[3];
+      float o3[3], db[RM], hb[RM];
+#pragma unroll
+      for (int kp = 0; kp < RM / 2; ++kp) {
+        db[2 * kp] = db2[kp].x;
+        db[2 * kp + 1] = db2[kp].y;
+        hb[2 * kp] = hb2[kp].x;
+        hb[2 * kp + 1] = hb2[kp].y;
+      }
       if constexpr (!DBL) {
         if (dvec) {
           edge_vec_grad<RM>(pl, v, acc, db, o3);

@@ -47,8 +47,8 @@ TPC_HD inline int wn_smem_bytes(int RM, int cpl, int nimax, int nmz_max, bool db
 }
 
 // ---- lane = edge (receiver adjoint streams, first and second order) --------
-// G, Gt : two chunk buffers of kWnChunk channels of G (and Gt), [u][k][m3] with
-//         row stride RM * n3max (zero where never staged)
+// G, Gt : two chunk buffers of kWnChunk channels of G (and Gt), [u][k/2][m3][k&1]
+//         with row stride RM * (2 l3 + 1) of the path (zero where never staged)
 // X, X1 : two chunk buffers of the 32 lanes' rows, [lane][u * n1 + m1] with row
 //         stride xs, xs / 4 odd: the 16-byte reads of 8 consecutive lanes fall
 //         into distinct bank quads

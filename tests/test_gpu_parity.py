@@ -174,6 +174,74 @@ def test_mace_full_size_sampled(T, gemm):
     assert rel(bw["dx"][ss], dx[ss]) < TOL[gemm]
 
 
+def _sub_csr(N, recv, mask):
+    """Receiver CSR over all N nodes holding only the masked edges (still receiver-sorted)."""
+    return np.concatenate([[0], np.cumsum(np.bincount(recv[mask], minlength=N))]).astype(np.int64)
+
+
+def _identity_ok(lhs_terms, rhs_terms):
+    """Scalar identity sum(lhs) = sum(rhs) of fp32 results: the fp32 bar (1e-5)
+    applied to the sums of absolute terms, the scale the rounding of every term
+    contributes to (the sums themselves cancel by orders of magnitude)."""
+    lhs = sum(float(t.sum()) for t in lhs_terms)
+    rhs = sum(float(t.sum()) for t in rhs_terms)
+    scale = sum(float(np.abs(t).sum()) for t in lhs_terms) + sum(float(np.abs(t).sum()) for t in rhs_terms)
+    return abs(lhs - rhs) <= TOL_FP32 * scale, (lhs, rhs, scale)
+
+
+@pytest.mark.parametrize("gemm", ["fp32"])
+def test_mace_full_size_dtheta_identity(T, gemm):
+    """dTheta at full size: out is linear in Theta, so <dTheta, D> = <g, out(x, D)>
+    for any direction D (both sides from the library; dTheta sums over all edges,
+    which the oracle cannot sample)."""
+    import torch
+    c = W.CONFIGS["mace"]
+    plan, prob, G, inp = make(T, c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], c["radial"],
+                              c["radial_params"], W.graph_for("mace", 0), seed=43, gemm=gemm)
+    rowptr, col, vec, x, th, g = inp
+    xd, thd, gd = dev(x, torch.float32), dev(th, torch.float32), dev(g, torch.float32)
+    dth = T.backward(plan, G, xd, thd, gd, want=("dtheta",))["dtheta"].double().cpu().numpy()
+    D = W.normal(th.shape, 44).astype(np.float32)
+    outD = T.forward(plan, G, xd, dev(D, torch.float32)).double().cpu().numpy()
+    ok, info = _identity_ok([dth * D.astype(np.float64)], [g * outD])
+    assert ok, info
+
+
+def test_mace_full_size_double_backward_sampled(T):
+    """The double backward of the bench step at full size (gg_x and gg_vec, no
+    gg_Theta; 3xTF32 Theta contractions).  d_g of sampled receivers and d_vec of
+    their edges depend only on those receivers' edges, d_x of sampled senders
+    only on their out-edges: the oracle computes them exactly on those sub-graphs.
+    d_Theta is checked through Psi's linearity in Theta:
+    <d_Theta, D> = <gg_x, dx(D)> + <gg_vec, dvec(D)>."""
+    import torch
+    c = W.CONFIGS["mace"]
+    plan, prob, G, inp = make(T, c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], c["radial"],
+                              c["radial_params"], W.graph_for("mace", 0), seed=45, gemm="fp32")
+    rowptr, col, vec, x, th, g = inp
+    r32 = lambda a: a.astype(np.float32).astype(np.float64)
+    ggx, ggv = r32(W.normal(x.shape, 46)), r32(W.normal(vec.shape, 47))
+    xd, thd, gd = dev(x, torch.float32), dev(th, torch.float32), dev(g, torch.float32)
+    ggxd, ggvd = dev(ggx, torch.float32), dev(ggv, torch.float32)
+    out = {k: v.double().cpu().numpy() for k, v in T.double_backward(plan, G, xd, thd, gd, ggxd, ggvd, None).items()}
+    N = len(rowptr) - 1
+    recv = np.repeat(np.arange(N), np.diff(rowptr))
+    rs = np.random.default_rng(2).choice(N, 20, replace=False)
+    em = np.isin(recv, rs)
+    ref = conv.double_backward(prob, _sub_csr(N, recv, em), col[em], vec[em], x, th, g, ggx, ggv[em], None)
+    assert rel(out["d_g"][rs], ref["d_g"][rs]) < TOL_FP32
+    assert rel(out["d_vec"][em], ref["d_vec"]) < TOL_FP32
+    ss = np.random.default_rng(3).choice(N, 12, replace=False)
+    sm = np.isin(col, ss)
+    ref2 = conv.double_backward(prob, _sub_csr(N, recv, sm), col[sm], vec[sm], x, th, g, ggx, ggv[sm], None)
+    assert rel(out["d_x"][ss], ref2["d_x"][ss]) < TOL_FP32
+    D = W.normal(th.shape, 48).astype(np.float32)
+    bw = T.backward(plan, G, xd, dev(D, torch.float32), gd, want=("dx", "dvec"))
+    ok, info = _identity_ok([out["d_theta"] * D.astype(np.float64)],
+                            [ggx * bw["dx"].double().cpu().numpy(), ggv * bw["dvec"].double().cpu().numpy()])
+    assert ok, info
+
+
 DBL_CASES = {
     "tiny_all": ("tiny", ("x", "v", "t")),
     "mixed_all": ("mixed_l3", ("x", "v", "t")),
