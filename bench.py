@@ -97,7 +97,9 @@ def work_model(T, plan):
         bw_r += 2 * nnz + ci * (2 * mnz + 2 * R * n3)             # M_e; M x, dT, db, Q += x (x) dT; C : Q
         bw_s += nnz + co * (mnz + R * n1)                         # M_e, M^T g, b (x) U
         db_a += 2 * nnz + ci * (3 * mnz + 3 * R * n3)
-        db_r += 4 * nnz + ci * (6 * mnz + 6 * R * n3)             # M, Md; 3 M-products, 3 Q updates; C : Qw, Qh
+        # M, Md; 3 M-products, 3 Q updates; C : Qw, Qh.  The step has no gg_Theta, so the
+        # G~ terms (b G~ into dX, G~ . T0 into wb; 2 R n3 per channel) are not part of it.
+        db_r += 4 * nnz + ci * (6 * mnz + 4 * R * n3)
         db_s += 2 * nnz + co * (2 * mnz + 3 * R * n1)
     return {"fwd_edge": fw, "bwd_edge_r": bw_r, "bwd_edge_s": bw_s, "dbl_edge_a": db_a, "dbl_edge_r": db_r,
             "dbl_edge_s": db_s}

@@ -19,7 +19,8 @@
 //   receiver, second order  A1 = sum_e b (M x1 + Md x) + bd (M x),  A0 = sum_e b (M x)
 //   sender,   second order  B1 = sum_e b (Md^T g) + bd (M^T g),     B0 = sum_e b (M^T g)
 // where Md, bd are the derivatives of M_e, b_e along the edge-vector
-// perturbation gg_vec_e and x1 = gg_x (terms with a missing input are zero).
+// perturbation gg_vec_e and x1 = gg_x (terms with a missing input are zero);
+// A0 / B0 are computed only by the P1 instantiations (when the caller needs them).
 #pragma once
 
 #include "async_copy.cuh"
@@ -82,7 +83,7 @@ __device__ __forceinline__ void ffma2_bcast(float2& a, float2 b, float t) { a = 
 // one path, all channel tiles of the warp's node.  The radial state is kept as
 // float2 pairs of consecutive radial indices, so the outer products b (x) T run
 // as paired FMAs; shared-memory strides are the path's own compile-time widths.
-template <int L1, int L2, int L3, int RM, int CPL, bool RECV, bool DBL>
+template <int L1, int L2, int L3, int RM, int CPL, bool RECV, bool DBL, bool P1>
 __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q, const WnLay& L, float* ws, int nl,
                                              int nc, int a0, int a1, const int* __restrict__ nbr,
                                              const int* __restrict__ perm, const float* __restrict__ vec,
@@ -93,7 +94,7 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
   constexpr int N2 = TR::N2, NMZ = TR::NMZ, NMP = (NMZ + 3) & ~3;
   constexpr int NI = RECV ? TR::N1 : TR::N3;  // staged floats per channel
   constexpr int NO = RECV ? TR::N3 : TR::N1;  // state floats per channel and radial index
-  constexpr int NPART = DBL ? 2 : 1;
+  constexpr int NPART = P1 ? 2 : 1;           // second order: A0 / B0 wanted
   constexpr int NK2 = RM / 2;                 // radial pairs
   constexpr int NACC = NPART * CPL * NK2 * NO;
   constexpr int XS = (32 * CPL * NI + 3) & ~3;  // staged row stride of this path (<= L.xs)
@@ -198,7 +199,7 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
 #pragma unroll
           for (int i = 0; i < NI; ++i) xv[i] = Xp[32 * NI * h + i];
           float2* a = acc + h * NK2 * NO;                 // part 0
-          float2* a1 = acc + (CPL + h) * NK2 * NO;        // part 1 (second order)
+          float2* a1 = acc + (P1 ? (CPL + h) * NK2 * NO : 0);  // part 1 (A0 / B0)
           if constexpr (!DBL) {
             float T[NO];
             if constexpr (RECV) apply_M<L1, L2, L3>(Mv, xv, T);
@@ -222,7 +223,7 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
               for (int i = 0; i < NO; ++i) {
                 ffma2_bcast(a[kp * NO + i], bd2[kp], T[i]);
                 ffma2_bcast(a[kp * NO + i], b2[kp], T1[i]);
-                ffma2_bcast(a1[kp * NO + i], b2[kp], T[i]);
+                if constexpr (P1) ffma2_bcast(a1[kp * NO + i], b2[kp], T[i]);
               }
           } else {
             float U[NO], U1[NO];
@@ -234,7 +235,7 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
               for (int i = 0; i < NO; ++i) {
                 ffma2_bcast(a[kp * NO + i], bd2[kp], U[i]);
                 ffma2_bcast(a[kp * NO + i], b2[kp], U1[i]);
-                ffma2_bcast(a1[kp * NO + i], b2[kp], U[i]);
+                if constexpr (P1) ffma2_bcast(a1[kp * NO + i], b2[kp], U[i]);
               }
           }
         }
@@ -273,7 +274,7 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
 // bodies and share their instructions in the instruction caches.
 // RECV: ptr = rowptr, nbr = col (edge id = CSR position); else ptr = s_rowptr,
 // nbr = s_recv, perm = sender-sorted position -> edge id.
-template <int RM, int LF, int CPL, bool RECV, bool DBL>
+template <int RM, int LF, int CPL, bool RECV, bool DBL, bool P1>
 __global__ void __launch_bounds__(32 * kWnWarps, 3)
     k_wn_stream(const __grid_constant__ DevPlan pl, int n0, int nc, const int* __restrict__ ptr,
                 const int* __restrict__ nbr, const int* __restrict__ perm, const float* __restrict__ vec,
@@ -293,8 +294,8 @@ __global__ void __launch_bounds__(32 * kWnWarps, 3)
 #define TPC_CASE(a, b, c)                                                                                        \
   case triple_id(a, b, c):                                                                                       \
     if constexpr (a <= LF && c <= LF)                                                                            \
-      wn_chan_path<a, b, c, RM, CPL, RECV, DBL>(pl, q, L, ws, nl, nc, a0, a1, nbr, perm, vec, ggv, src, src1, out, \
-                                                out0);                                                           \
+      wn_chan_path<a, b, c, RM, CPL, RECV, DBL, P1>(pl, q, L, ws, nl, nc, a0, a1, nbr, perm, vec, ggv, src, src1, \
+                                                    out, out0);                                                  \
     break;
     TPC_FOR_EACH_TRIPLE(TPC_CASE)
 #undef TPC_CASE

@@ -67,8 +67,8 @@ __host__ __device__ constexpr int g_slot(int k, int m3) {
   return ((k >> 1) * N3 + m3) * 2 + (k & 1);
 }
 
-// one path of one 32-edge batch
-template <int L1, int L2, int L3, int RM, bool DBL>
+// one path of one 32-edge batch (GT: the second order has a Gt operand)
+template <int L1, int L2, int L3, int RM, bool DBL, bool GT>
 __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, const WnaLay& L, float* ws, int rl,
                                          int nc, int nb, int myrow, const float* __restrict__ x,
                                          const float* __restrict__ x1, const float* __restrict__ G,
@@ -111,7 +111,8 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
   const int c = q.c_in, R = pl.R;
   const int nch = c / CH;  // channel counts are multiples of four on this path
   const int Kb = pl.Kb[q.i3];
-  const bool has_t = DBL && Gt != nullptr, has_x1 = DBL && x1 != nullptr;
+  constexpr bool has_t = DBL && GT;
+  const bool has_x1 = DBL && x1 != nullptr;
   // this lane's G elements of a chunk: source offset (relative to channel u0)
   // and shared slot, the same for every chunk of the path
   const float* Gp = G + size_t(nc) * pl.a_pref[q.i3] + size_t(rl) * N3 * Kb + q.koff;
@@ -133,7 +134,7 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
     for (int it = 0; it < NIT; ++it) {
       if (gsrc[it] >= 0) {
         ac_copy4(sG + gdst[it], Gp + u0 + gsrc[it]);
-        if (has_t) ac_copy4(sGt + gdst[it], Gtp + u0 + gsrc[it]);
+        if constexpr (has_t) ac_copy4(sGt + gdst[it], Gtp + u0 + gsrc[it]);
       }
     }
     // the batch's rows, N1 16-byte pieces each, copied by the whole warp (coalesced)
@@ -199,25 +200,28 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
         float2 dG2[N3], dX2[N3];
 #pragma unroll
         for (int i = 0; i < N3; ++i) dG2[i] = dX2[i] = make_float2(0.f, 0.f);
-        // G and Gt rows in KH slices of radial pairs (bounds the live registers)
+        // G (and Gt) rows in KH slices of radial pairs (bounds the live registers)
         constexpr int KH = NK2 >= 4 ? 2 : 1, KS = NK2 / KH;  // KS pairs per slice
 #pragma unroll
         for (int kh = 0; kh < KH; ++kh) {
-          float2 g2[KS * N3], gt2[KS * N3];
+          float2 g2[KS * N3], gt2[GT ? KS * N3 : 1];
           lds_f2<KS * N3>(sG + t * GW + 2 * kh * KS * N3, g2);
-          lds_f2<KS * N3>(sGt + t * GW + 2 * kh * KS * N3, gt2);
+          if constexpr (GT) lds_f2<KS * N3>(sGt + t * GW + 2 * kh * KS * N3, gt2);
 #pragma unroll
           for (int kk = 0; kk < KS; ++kk) {
             const int kp = kh * KS + kk;
 #pragma unroll
             for (int i = 0; i < N3; ++i) {
-              const float2 g = g2[kk * N3 + i], gt = gt2[kk * N3 + i];
+              const float2 g = g2[kk * N3 + i];
               dG2[i] = __ffma2_rn(b2[kp], g, dG2[i]);
               dX2[i] = __ffma2_rn(bd2[kp], g, dX2[i]);
-              dX2[i] = __ffma2_rn(b2[kp], gt, dX2[i]);
-              db[kp] = __ffma2_rn(gt, make_float2(T[i], T[i]), db[kp]);
               db[kp] = __ffma2_rn(g, make_float2(T12[i], T12[i]), db[kp]);
               hb[kp] = __ffma2_rn(g, make_float2(T[i], T[i]), hb[kp]);
+              if constexpr (GT) {
+                const float2 gt = gt2[kk * N3 + i];
+                dX2[i] = __ffma2_rn(b2[kp], gt, dX2[i]);
+                db[kp] = __ffma2_rn(gt, make_float2(T[i], T[i]), db[kp]);
+              }
             }
           }
         }
@@ -257,8 +261,9 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
 // instruction caches; every warp runs the CTA's largest batch count, the ones
 // with fewer batches (or no node) joining the barriers without work.
 // First order writes dvec (and, when given, dY [E][n_sh], db [E][R]); second
-// order writes dvec.  x1 / Gt / ggv may be null (their terms vanish).
-template <int RM, int LF, bool DBL>
+// order writes dvec.  x1 / ggv may be null (their terms vanish); Gt is used
+// exactly when GT.
+template <int RM, int LF, bool DBL, bool GT>
 __global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
     k_wn_adj(const __grid_constant__ DevPlan pl, int r0, int nc, const int* __restrict__ rowptr,
              const int* __restrict__ col, const float* __restrict__ vec, const float* __restrict__ ggv,
@@ -332,7 +337,7 @@ __global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
 #define TPC_CASE(a, b, c)                                                                                 \
   case triple_id(a, b, c):                                                                                \
     if constexpr (a <= LF && c <= LF)                                                                     \
-      wna_path<a, b, c, RM, DBL>(pl, q, L, ws, rl, nc, nb, myrow, x, x1, G, Gt, db2, hb2);                  \
+      wna_path<a, b, c, RM, DBL, GT>(pl, q, L, ws, rl, nc, nb, myrow, x, x1, G, Gt, db2, hb2);                  \
     break;
           TPC_FOR_EACH_TRIPLE(TPC_CASE)
 #undef TPC_CASE

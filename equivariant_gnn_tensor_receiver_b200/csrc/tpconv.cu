@@ -520,7 +520,8 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
       const int nc = int(std::min<int64_t>(Nc, N - r0));
       {
         PhaseScope ps(TPCONV_PHASE_DBL_EDGE_A, s);
-        if (TPC_WN_CALL(d, launch_wn_dbla, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, A1, A0, s))
+        if (TPC_WN_CALL(d, launch_wn_dbla, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, A1,
+                        has_t ? A0 : nullptr, s))
           return TPCONV_ERR_CUDA;
         note(TPCONV_PHASE_DBL_EDGE_A, 1);
       }
@@ -566,7 +567,8 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
       const int nc = int(std::min<int64_t>(Nc, N - s0));
       {
         PhaseScope ps(TPCONV_PHASE_DBL_EDGE_S, s);
-        if (TPC_WN_CALL(d, launch_wn_dbls, d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, gg_vec, g, B1, B0, s))
+        if (TPC_WN_CALL(d, launch_wn_dbls, d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, gg_vec, g, B1,
+                        (has_x1 || has_t) ? B0 : nullptr, s))
           return TPCONV_ERR_CUDA;
         note(TPCONV_PHASE_DBL_EDGE_S, 1);
       }
