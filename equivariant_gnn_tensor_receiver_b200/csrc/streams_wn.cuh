@@ -275,7 +275,7 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
 // RECV: ptr = rowptr, nbr = col (edge id = CSR position); else ptr = s_rowptr,
 // nbr = s_recv, perm = sender-sorted position -> edge id.
 template <int RM, int LF, int CPL, bool RECV, bool DBL, bool P1>
-__global__ void __launch_bounds__(32 * kWnWarps, 3)
+__global__ void __launch_bounds__(32 * kWnWarps, DBL && RECV ? 3 : 4)
     k_wn_stream(const __grid_constant__ DevPlan pl, int n0, int nc, const int* __restrict__ ptr,
                 const int* __restrict__ nbr, const int* __restrict__ perm, const float* __restrict__ vec,
                 const float* __restrict__ ggv, const float* __restrict__ src, const float* __restrict__ src1,
