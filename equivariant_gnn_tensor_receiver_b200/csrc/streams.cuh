@@ -113,6 +113,57 @@ __device__ __forceinline__ void apply_Mt(const float* __restrict__ Mj, const flo
   });
 }
 
+// Paired forms for a coupling matrix and its derivative stored side by side,
+// MM[mi] = (M[mi], Md[mi]): one paired FMA applies both.
+// (T[m3], Td[m3]) = sum_m1 (M, Md)[m1][m3] x[m1]
+template <int L1, int L2, int L3>
+__device__ __forceinline__ void apply_M2(const float2* MM, const float* xv, float2* TT) {
+  using TR = Tri<L1, L2, L3>;
+#pragma unroll
+  for (int i3 = 0; i3 < TR::N3; ++i3) TT[i3] = make_float2(0.f, 0.f);
+  sfor<TR::N1>([&](auto I1) {
+    sfor<TR::N3>([&](auto I3) {
+      constexpr int i1 = decltype(I1)::value, i3 = decltype(I3)::value;
+      if constexpr (TR::tab.m[i1][i3]) {
+        constexpr int mi = TR::tab.mi[i1][i3];
+        TT[i3] = __ffma2_rn(MM[mi], make_float2(xv[i1], xv[i1]), TT[i3]);
+      }
+    });
+  });
+}
+// (U[m1], Ud[m1]) = sum_m3 (M, Md)[m1][m3] y[m3]
+template <int L1, int L2, int L3>
+__device__ __forceinline__ void apply_Mt2(const float2* MM, const float* yv, float2* UU) {
+  using TR = Tri<L1, L2, L3>;
+#pragma unroll
+  for (int i1 = 0; i1 < TR::N1; ++i1) UU[i1] = make_float2(0.f, 0.f);
+  sfor<TR::N1>([&](auto I1) {
+    sfor<TR::N3>([&](auto I3) {
+      constexpr int i1 = decltype(I1)::value, i3 = decltype(I3)::value;
+      if constexpr (TR::tab.m[i1][i3]) {
+        constexpr int mi = TR::tab.mi[i1][i3];
+        UU[i1] = __ffma2_rn(MM[mi], make_float2(yv[i3], yv[i3]), UU[i1]);
+      }
+    });
+  });
+}
+// T[m3] = sum_m1 M[m1][m3] x[m1] with M the first members of MM
+template <int L1, int L2, int L3>
+__device__ __forceinline__ void apply_M_first(const float2* MM, const float* xv, float* T) {
+  using TR = Tri<L1, L2, L3>;
+#pragma unroll
+  for (int i3 = 0; i3 < TR::N3; ++i3) T[i3] = 0.f;
+  sfor<TR::N1>([&](auto I1) {
+    sfor<TR::N3>([&](auto I3) {
+      constexpr int i1 = decltype(I1)::value, i3 = decltype(I3)::value;
+      if constexpr (TR::tab.m[i1][i3]) {
+        constexpr int mi = TR::tab.mi[i1][i3];
+        T[i3] = fmaf(MM[mi].x, xv[i1], T[i3]);
+      }
+    });
+  });
+}
+
 // out[m2] = sum_{m1,m3} C[m1,m2,m3] a[m1] c[m3]
 template <int L1, int L2, int L3>
 __device__ __forceinline__ void cg_contract_13(const float* a, const float* c, float* out) {

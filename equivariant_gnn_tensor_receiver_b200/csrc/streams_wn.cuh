@@ -107,7 +107,6 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
   const int nsb = (ne + kWnSub - 1) / kWnSub;
   const bool two = DBL && RECV && src1 != nullptr;
   float* sM = ws + L.M;
-  float* sMd = ws + L.Md;
   float* sB = ws + L.B;
   float* sBd = ws + L.Bd;
   float* sX = ws + L.X;
@@ -161,11 +160,19 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
           float Y[N2], Yd[N2], b[RM], bd[RM], Mrow[NMP];
           wn_geometry<L2, RM, DBL>(pl, vec, ggv, e, Y, Yd, b, bd);
           wn_coupling<L1, L2, L3, NMP>(Y, Mrow);
-          sts_vec<NMP>(sM + lane * NMP, Mrow);
           sts_vec<RM>(sB + lane * RM, b);
-          if constexpr (DBL) {
-            wn_coupling<L1, L2, L3, NMP>(Yd, Mrow);
-            sts_vec<NMP>(sMd + lane * NMP, Mrow);
+          if constexpr (!DBL) {
+            sts_vec<NMP>(sM + lane * NMP, Mrow);
+          } else {
+            // (M, Md) side by side: [edge][mi][2] over the M and Md regions
+            float Mdrow[NMP], MM[2 * NMP];
+            wn_coupling<L1, L2, L3, NMP>(Yd, Mdrow);
+#pragma unroll
+            for (int i = 0; i < NMP; ++i) {
+              MM[2 * i] = Mrow[i];
+              MM[2 * i + 1] = Mdrow[i];
+            }
+            sts_vec<2 * NMP>(sM + lane * 2 * NMP, MM);
             sts_vec<RM>(sBd + lane * RM, bd);
           }
         }
@@ -176,23 +183,20 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
       ac_wait<1>();
       __syncwarp();
       const int nb = min(kWnSub, ne - j0);
-      const float* Mp = sM + (j0 & 31) * NMP;
-      const float* Mdp = sMd + (j0 & 31) * NMP;
+      const float* Mp = sM + (j0 & 31) * (DBL ? 2 * NMP : NMP);
       const float* Bp = sB + (j0 & 31) * RM;
       const float* Bdp = sBd + (j0 & 31) * RM;
       const float* Xp = sX + (sb & 1) * BUF + lane * NI;
       const float* X1p = sX1 + (sb & 1) * BUF + lane * NI;
-      for (int jj = 0; jj < nb; ++jj, Mp += NMP, Mdp += NMP, Bp += RM, Bdp += RM, Xp += XS, X1p += XS) {
-        float Mv[NMP];
+      for (int jj = 0; jj < nb; ++jj, Mp += (DBL ? 2 * NMP : NMP), Bp += RM, Bdp += RM, Xp += XS, X1p += XS) {
+        float Mv[DBL ? 1 : NMP];
+        float2 MM[DBL ? NMP : 1];  // second order: (M, Md) pairs
         float2 b2[NK2];
-        lds_vec<NMP>(Mp, Mv);
+        if constexpr (!DBL) lds_vec<NMP>(Mp, Mv);
+        else lds_f2<NMP>(Mp, MM);
         lds_f2<NK2>(Bp, b2);
-        float Mdv[DBL ? NMP : 1];
         float2 bd2[DBL ? NK2 : 1];
-        if constexpr (DBL) {
-          lds_vec<NMP>(Mdp, Mdv);
-          lds_f2<NK2>(Bdp, bd2);
-        }
+        if constexpr (DBL) lds_f2<NK2>(Bdp, bd2);
 #pragma unroll
         for (int h = 0; h < CPL; ++h) {
           float xv[NI];
@@ -209,14 +213,17 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
 #pragma unroll
               for (int i = 0; i < NO; ++i) ffma2_bcast(a[kp * NO + i], b2[kp], T[i]);
           } else if constexpr (RECV) {
-            float x1v[NI], T[NO], T1[NO], T2[NO];
+            float x1v[NI], T[NO], T1[NO];
+            float2 TT[NO];  // (M x, Md x)
 #pragma unroll
             for (int i = 0; i < NI; ++i) x1v[i] = two ? X1p[i] : 0.f;
-            apply_M<L1, L2, L3>(Mv, xv, T);
-            apply_M<L1, L2, L3>(Mv, x1v, T1);
-            apply_M<L1, L2, L3>(Mdv, xv, T2);
+            apply_M2<L1, L2, L3>(MM, xv, TT);
+            apply_M_first<L1, L2, L3>(MM, x1v, T1);
 #pragma unroll
-            for (int i = 0; i < NO; ++i) T1[i] += T2[i];
+            for (int i = 0; i < NO; ++i) {
+              T[i] = TT[i].x;
+              T1[i] += TT[i].y;
+            }
 #pragma unroll
             for (int kp = 0; kp < NK2; ++kp)
 #pragma unroll
@@ -226,9 +233,14 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
                 if constexpr (P1) ffma2_bcast(a1[kp * NO + i], b2[kp], T[i]);
               }
           } else {
+            float2 UU[NO];  // (M^T g, Md^T g)
+            apply_Mt2<L1, L2, L3>(MM, xv, UU);
             float U[NO], U1[NO];
-            apply_Mt<L1, L2, L3>(Mv, xv, U);
-            apply_Mt<L1, L2, L3>(Mdv, xv, U1);
+#pragma unroll
+            for (int i = 0; i < NO; ++i) {
+              U[i] = UU[i].x;
+              U1[i] = UU[i].y;
+            }
 #pragma unroll
             for (int kp = 0; kp < NK2; ++kp)
 #pragma unroll

@@ -42,6 +42,35 @@ __device__ __forceinline__ void outer_Q(const float* a, const float* c, float* Q
   });
 }
 
+// (Q[mi], Q'[mi]) += (a[m1], a'[m1]) c[m3] on the structural nonzeros
+template <int L1, int L2, int L3>
+__device__ __forceinline__ void outer_Q2(const float* a, const float* a2, const float* c, float2* QQ) {
+  using TR = Tri<L1, L2, L3>;
+  sfor<TR::N1>([&](auto I1) {
+    sfor<TR::N3>([&](auto I3) {
+      constexpr int i1 = decltype(I1)::value, i3 = decltype(I3)::value;
+      if constexpr (TR::tab.m[i1][i3]) {
+        constexpr int mi = TR::tab.mi[i1][i3];
+        QQ[mi] = __ffma2_rn(make_float2(a[i1], a2[i1]), make_float2(c[i3], c[i3]), QQ[mi]);
+      }
+    });
+  });
+}
+// Q[mi] += a[m1] c[m3] into the first members of QQ
+template <int L1, int L2, int L3>
+__device__ __forceinline__ void outer_Q_first(const float* a, const float* c, float2* QQ) {
+  using TR = Tri<L1, L2, L3>;
+  sfor<TR::N1>([&](auto I1) {
+    sfor<TR::N3>([&](auto I3) {
+      constexpr int i1 = decltype(I1)::value, i3 = decltype(I3)::value;
+      if constexpr (TR::tab.m[i1][i3]) {
+        constexpr int mi = TR::tab.mi[i1][i3];
+        QQ[mi].x = fmaf(a[i1], c[i3], QQ[mi].x);
+      }
+    });
+  });
+}
+
 // out[m2] += sum_{m1,m3} C[m1,m2,m3] Q[m1][m3]
 template <int L1, int L2, int L3>
 __device__ __forceinline__ void contract_Q(const float* Q, float* out) {
@@ -80,25 +109,28 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
   constexpr int NIT = (GW * CH + 31) / 32;  // G elements per lane and chunk (upper bound)
   const int lane = lane_id();
   const float* geo = ws + L.Geo + lane * L.geos;
-  float Mv[NMZ];
-  float2 b2[NK2];
+  // first order: M in Mv; second order: (M, Md) side by side in MM (paired FMAs);
+  // accumulators Q (second order: Qw) and Qh
+  float Mv[DBL ? 1 : NMZ];
+  float2 MM[DBL ? NMZ : 1];
+  float2 b2[NK2], bd2[DBL ? NK2 : 1];
   {
-    float Y[N2];
+    float Y[N2], Mrow[NMZ];
 #pragma unroll
     for (int i = 0; i < N2; ++i) Y[i] = geo[L2 * L2 + i];
-    coupling_row<L1, L2, L3>(Y, Mv);
+    coupling_row<L1, L2, L3>(Y, DBL ? Mrow : Mv);
 #pragma unroll
     for (int kp = 0; kp < NK2; ++kp) b2[kp] = make_float2(geo[16 + 2 * kp], geo[17 + 2 * kp]);
-  }
-  float Mdv[DBL ? NMZ : 1];
-  float2 bd2[DBL ? NK2 : 1];
-  if constexpr (DBL) {
-    float Y[N2];
+    if constexpr (DBL) {
+      float Mdrow[NMZ];
 #pragma unroll
-    for (int i = 0; i < N2; ++i) Y[i] = geo[16 + RM + L2 * L2 + i];
-    coupling_row<L1, L2, L3>(Y, Mdv);
+      for (int i = 0; i < N2; ++i) Y[i] = geo[16 + RM + L2 * L2 + i];
+      coupling_row<L1, L2, L3>(Y, Mdrow);
 #pragma unroll
-    for (int kp = 0; kp < NK2; ++kp) bd2[kp] = make_float2(geo[32 + RM + 2 * kp], geo[33 + RM + 2 * kp]);
+      for (int i = 0; i < NMZ; ++i) MM[i] = make_float2(Mrow[i], Mdrow[i]);
+#pragma unroll
+      for (int kp = 0; kp < NK2; ++kp) bd2[kp] = make_float2(geo[32 + RM + 2 * kp], geo[33 + RM + 2 * kp]);
+    }
   }
   float Q[NMZ], Qh[DBL ? NMZ : 1];
 #pragma unroll
@@ -170,9 +202,9 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
 #pragma unroll
     for (int t = 0; t < CH; ++t) {
       const float* xv = xg + t * N1;
-      float T[N3];
-      apply_M<L1, L2, L3>(Mv, xv, T);
       if constexpr (!DBL) {
+        float T[N3];
+        apply_M<L1, L2, L3>(Mv, xv, T);
         float2 g2[NK2 * N3];
         lds_f2<NK2 * N3>(sG + t * GW, g2);
         float2 dT2[N3];
@@ -192,11 +224,15 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
         outer_Q<L1, L2, L3>(xv, dT, Q);
       } else {
         const float* x1v = x1g + t * N1;
-        float T12[N3], Tb[N3];
-        apply_M<L1, L2, L3>(Mv, x1v, T12);
-        apply_M<L1, L2, L3>(Mdv, xv, Tb);
+        float2 TT[N3];  // (M x, Md x)
+        apply_M2<L1, L2, L3>(MM, xv, TT);
+        float T[N3], T12[N3];
+        apply_M_first<L1, L2, L3>(MM, x1v, T12);
 #pragma unroll
-        for (int i = 0; i < N3; ++i) T12[i] += Tb[i];
+        for (int i = 0; i < N3; ++i) {
+          T[i] = TT[i].x;
+          T12[i] += TT[i].y;
+        }
         float2 dG2[N3], dX2[N3];
 #pragma unroll
         for (int i = 0; i < N3; ++i) dG2[i] = dX2[i] = make_float2(0.f, 0.f);
