@@ -96,7 +96,7 @@ def work_model(T, plan):
         fw += nnz + ci * (mnz + R * n3)                           # M_e, M x, b (x) T
         bw_r += 2 * nnz + ci * (2 * mnz + 2 * R * n3)             # M_e; M x, dT, db, Q += x (x) dT; C : Q
         bw_s += nnz + co * (mnz + R * n1)                         # M_e, M^T g, b (x) U
-        db_a += 2 * nnz + ci * (3 * mnz + 3 * R * n3)
+        db_a += 2 * nnz + ci * (3 * mnz + 2 * R * n3)             # A1 only: A0 serves gg_Theta, absent here
         # M, Md; 3 M-products, 3 Q updates; C : Qw, Qh.  The step has no gg_Theta, so the
         # G~ terms (b G~ into dX, G~ . T0 into wb; 2 R n3 per channel) are not part of it.
         db_r += 4 * nnz + ci * (6 * mnz + 4 * R * n3)
