@@ -33,8 +33,22 @@ sys.path.insert(0, ROOT)
 
 import workloads as W  # noqa: E402
 
-WORKLOAD = ("mace-like layer: 4096 atoms, periodic cube at 0.1 atoms/A^3, 5 A radius graph, "
-            "64x0e+64x1o+64x2e -> 64x0e+64x1o+64x2e, SH l<=3, R=8 Bessel")
+WORKLOADS = {
+    "mace": ("mace-like layer: 4096 atoms, periodic cube at 0.1 atoms/A^3, 5 A radius graph, "
+             "64x0e+64x1o+64x2e -> 64x0e+64x1o+64x2e, SH l<=3, R=8 Bessel"),
+    "capacity": ("capacity run of the mace-like layer: 1222309 atoms, periodic cube at 0.1 atoms/A^3 "
+                 "(side 230.35 A), 5 A radius graph (~64 M edges), 64x0e+64x1o+64x2e, SH l<=3, R=8 Bessel; "
+                 "receiver chunks of the workspace cap"),
+    "sweep": ("edge-scaling sweep: 20000 nodes, periodic cube sized for mean degree {d:g}, 5 A radius graph, "
+              "32x0e+32x1o+32x2e, SH l<=2, R=8 Bessel"),
+    "wide": ("wide operator: 8192 nodes, mean degree 32, 5 A radius graph, 128x0e+128x1o+128x2e+128x3o, "
+             "SH l<=3, R=8 Bessel"),
+    "tiny": "tiny: 64 nodes, 512 random edges, 8x0e+8x1o, SH l<=2, R=4 Gaussian",
+}
+
+
+def workload(args):
+    return WORKLOADS[args.config].format(d=args.degree or 25)
 METRIC = "edges/s (fwd + bwd + double bwd step)"
 L2_BYTES = 126 * 1024 * 1024
 FP32_LANES_PER_SM = 128
@@ -50,6 +64,9 @@ def parse():
     ap.add_argument("--config", default="mace")
     ap.add_argument("--gemm", default="fp32", choices=["fp32", "tf32", "simt"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--degree", type=float, default=None, help="mean degree of the sweep workload")
+    ap.add_argument("--workspace-cap", type=int, default=None,
+                    help="bytes of node-side state per receiver chunk (default: none; 8 GiB for capacity)")
     return ap.parse_args()
 
 
@@ -170,9 +187,13 @@ def oracle_sample(cfg, graph, n_recv, seed=100):
     prob = conv.Problem(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], c["radial"],
                         tuple(c["radial_params"]))
     rowptr, col, vec = graph
-    N = len(rowptr) - 1
     e1 = int(rowptr[n_recv])
     rp = np.asarray(rowptr[:n_recv + 1], dtype=np.int64)
+    # only the sample's receivers (first, keeping their numbers) and senders hold features
+    nodes = np.unique(np.concatenate([np.arange(n_recv), np.asarray(col[:e1], dtype=np.int64)]))
+    col = np.searchsorted(nodes, np.asarray(col[:e1], dtype=np.int64)).astype(np.int32)
+    vec = vec[:e1]
+    N = len(nodes)
     x = W.normal((N, prob.dim_in), seed)
     th = W.theta([(prob.R * p.c_in * p.c_out, 1 / np.sqrt(prob.R * p.c_in)) for p in prob.paths], seed + 1)
     g = np.zeros((n_recv, prob.dim_out))
@@ -229,7 +250,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "edges/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "sample": f"edges of the first {n_recv} receivers ({e} edges)"},
+            "config": {"workload": workload(args), "sample": f"edges of the first {n_recv} receivers ({e} edges)"},
             "cpu_baseline": {"value": v, "unit": "edges/s", "cores": cores, "kind": "oracle",
                              "sample": f"fp64 numpy oracle, conventional schedule, {e} edges per step"},
             "e2e": {"value": v, "unit": "edges/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -252,10 +273,11 @@ def run_ours(args):
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
     c = W.CONFIGS[args.config]
-    rowptr, col, vec = W.graph_for(args.config, rank)
+    rowptr, col, vec = W.graph_for(args.config, rank, args.degree)
     N, E = len(rowptr) - 1, len(col)
+    cap = args.workspace_cap if args.workspace_cap is not None else (8 << 30 if args.config == "capacity" else 0)
     plan = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], radial=c["radial"],
-                  radial_params=c["radial_params"], gemm=args.gemm)
+                  radial_params=c["radial_params"], gemm=args.gemm, workspace_cap=cap)
     f32 = torch.float32
     pin = lambda a, dt=f32: torch.as_tensor(np.ascontiguousarray(a), dtype=dt).pin_memory()
     host = {
@@ -392,7 +414,7 @@ def run_ours(args):
             "metric": METRIC, "value": job_value, "unit": "edges/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": step_ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "nodes_per_gpu": N, "edges_per_gpu": E, "gemm": args.gemm,
+            "config": {"workload": workload(args), "workspace_cap": cap, "nodes_per_gpu": N, "edges_per_gpu": E, "gemm": args.gemm,
                        "step": "graph transpose + fwd + bwd(dx,dTheta,dvec) + double bwd(gg_x,gg_vec)",
                        "l2": "256 MiB buffer zeroed before every timed step, outside the events",
                        "parallelism": f"{world} independent replicas (one graph per rank)"},

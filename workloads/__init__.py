@@ -20,6 +20,9 @@ Workload recipes (one per configuration of the layer):
     wide   N=8192, mean degree 32, 5 A cutoff; 128x0e+128x1o+128x2e+128x3o,
            SH l<=3, R=8 Bessel.
     dbl    graph and irreps of ``mace`` (double backward).
+    capacity  irreps of ``mace`` on 1 222 309 atoms at the same density and
+           cutoff (cube side 230.35 A): about 64 M edges, node-side state of
+           107.6 GB if held at once, so it runs in receiver chunks.
 Features x, cotangents g, gg ~ N(0, 1); Theta ~ N(0, std^2) with
 std = 1/sqrt(R * C_in) per path block.
 """
@@ -41,6 +44,8 @@ CONFIGS = {
                  l_sh_max=3, R=8, radial="bessel", radial_params=(5.0,)),
 }
 CONFIGS["dbl"] = dict(CONFIGS["mace"])
+CONFIGS["capacity"] = dict(CONFIGS["mace"])
+CAPACITY_ATOMS = 1222309
 
 
 def rng(seed: int) -> np.random.Generator:
@@ -146,4 +151,6 @@ def graph_for(name: str, seed: int, degree: float | None = None):
         return radius_graph(20000, box_for_degree(20000, 5.0, degree or 25), 5.0, seed)
     if name == "wide":
         return radius_graph(8192, box_for_degree(8192, 5.0, 32), 5.0, seed)
+    if name == "capacity":
+        return radius_graph(CAPACITY_ATOMS, (CAPACITY_ATOMS / 0.1) ** (1.0 / 3.0), 5.0, seed)
     raise ValueError(name)
