@@ -10,9 +10,9 @@ double backward.  All arithmetic runs in the CUDA library ``libtpconv.so``
 from ._lib import (GEMM, OP_BACKWARD, OP_DOUBLE_BACKWARD, OP_FORWARD, OP_TRANSPOSE, Plan, TPConvError,
                    exported_names, lib, tpconv_backward, tpconv_cg_coefficients, tpconv_double_backward,
                    tpconv_forward, tpconv_graph_transpose, tpconv_plan_create, tpconv_workspace_size)
-from .api import Graph, backward, double_backward, forward, workspace
+from .api import Graph, TPConv, backward, double_backward, forward, workspace
 
-__all__ = ["Plan", "Graph", "TPConvError", "forward", "backward", "double_backward", "workspace", "lib",
+__all__ = ["Plan", "Graph", "TPConv", "TPConvError", "forward", "backward", "double_backward", "workspace", "lib",
            "exported_names", "tpconv_plan_create", "tpconv_forward", "tpconv_backward", "tpconv_double_backward",
            "tpconv_graph_transpose", "tpconv_workspace_size", "tpconv_cg_coefficients", "GEMM", "OP_FORWARD",
            "OP_BACKWARD", "OP_DOUBLE_BACKWARD", "OP_TRANSPOSE"]

@@ -85,3 +85,60 @@ def double_backward(plan, graph: Graph, x, theta, g, gg_x=None, gg_vec=None, gg_
                              graph.edge_vec, x, theta, g, gg_x, gg_vec, gg_theta, outs["d_g"], outs["d_x"],
                              outs["d_vec"], outs["d_theta"], ws, stream)
     return {k: v for k, v in outs.items() if v is not None}
+
+
+# ---------------------------------------------------------------------------
+# torch autograd glue: every product below runs in the library (C ABI); the
+# Functions only route tensors.  d(out)/d(x, theta, edge_vec) is the library's
+# backward; the backward of that backward is its double backward, so forces
+# (-d energy / d positions) can themselves be differentiated.
+# ---------------------------------------------------------------------------
+class _ConvFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, theta, edge_vec, plan, graph):
+        ctx.plan, ctx.graph = plan, graph
+        ctx.save_for_backward(x, theta, edge_vec)
+        return forward(plan, graph, x.contiguous(), theta.contiguous())
+
+    @staticmethod
+    def backward(ctx, g):
+        x, theta, edge_vec = ctx.saved_tensors
+        dx, dtheta, dvec = _ConvBwdFn.apply(x, theta, edge_vec, g.contiguous(), ctx.plan, ctx.graph)
+        return dx, dtheta, dvec, None, None
+
+
+class _ConvBwdFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, theta, edge_vec, g, plan, graph):
+        ctx.plan, ctx.graph = plan, graph
+        ctx.save_for_backward(x, theta, edge_vec, g)
+        r = backward(plan, graph, x.contiguous(), theta.contiguous(), g, want=("dx", "dtheta", "dvec"))
+        return r["dx"], r["dtheta"], r["dvec"]
+
+    @staticmethod
+    def backward(ctx, gg_x, gg_theta, gg_vec):
+        x, theta, edge_vec, g = ctx.saved_tensors
+        c = lambda t: None if t is None else t.contiguous()
+        r = double_backward(ctx.plan, ctx.graph, x.contiguous(), theta.contiguous(), g, c(gg_x), c(gg_vec),
+                            c(gg_theta))
+        return r["d_x"], r["d_theta"], r["d_vec"], r["d_g"], None, None
+
+
+class TPConv(torch.nn.Module):
+    """The streaming CG tensor-product convolution as a torch module.
+
+    Holds Theta ([P][R][C_in][C_out], one normal block per path with standard
+    deviation 1/sqrt(R C_in)) as a parameter; ``forward(x, graph)`` returns
+    out[N][dim_out] for the receiver-sorted ``Graph`` (its ``edge_vec`` may
+    require grad).  Differentiable twice in x, Theta and the edge vectors.
+    """
+
+    def __init__(self, irreps_in, l_sh_max, irreps_out, R, device="cuda", **plan_options):
+        super().__init__()
+        self.plan = L.Plan(irreps_in, l_sh_max, irreps_out, R, **plan_options)
+        blocks = [torch.randn(self.plan.R * p["c_in"] * p["c_out"]) / (self.plan.R * p["c_in"]) ** 0.5
+                  for p in self.plan.paths]
+        self.theta = torch.nn.Parameter(torch.cat(blocks).to(device=device, dtype=torch.float32))
+
+    def forward(self, x, graph: Graph):
+        return _ConvFn.apply(x, self.theta, graph.edge_vec, self.plan, graph)

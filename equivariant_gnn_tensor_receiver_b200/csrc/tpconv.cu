@@ -279,6 +279,48 @@ cudaError_t node_mix_sender(const tpconv_plan* plan, int s0, int nc, const float
   return cudaSuccess;
 }
 
+// ---- validate mode: the graph is checked on the device before any stream runs ----
+__device__ int g_graph_error;
+
+// rowptr non-decreasing from 0 to E, senders in [0, N), edge vectors finite and nonzero
+__global__ void k_validate_graph(int64_t N, int64_t E, const int32_t* __restrict__ rowptr,
+                                 const int32_t* __restrict__ col, const float* __restrict__ vec) {
+  int bad = 0;
+  const int64_t n = N + 1 > E ? N + 1 : E;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    if (i < N && rowptr[i] > rowptr[i + 1]) bad = 1;
+    if (i == 0 && (rowptr[0] != 0 || int64_t(rowptr[N]) != E)) bad = 1;
+    if (i < E) {
+      const int32_t c = col[i];
+      if (c < 0 || int64_t(c) >= N) bad = 1;
+      if (vec) {
+        const float x = vec[3 * i], y = vec[3 * i + 1], z = vec[3 * i + 2];
+        const float r2 = x * x + y * y + z * z;
+        if (!(r2 > 0.f) || !isfinite(r2)) bad = 1;
+      }
+    }
+  }
+  if (bad) atomicOr(&g_graph_error, 1);
+}
+
+// With plan->opt.validate set: check the receiver CSR (and edge vectors) and
+// wait for the answer; TPCONV_ERR_GRAPH_INVALID stops the call before any
+// kernel reads the graph.  Otherwise a no-op.
+int validate_graph(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t* rowptr, const int32_t* col,
+                   const float* vec, cudaStream_t s) {
+  if (!plan->opt.validate) return TPCONV_OK;
+  const int zero = 0;
+  int flag = 0;
+  if (cudaMemcpyToSymbolAsync(g_graph_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s)) return TPCONV_ERR_CUDA;
+  const int64_t n = std::max<int64_t>(N + 1, E);
+  const unsigned blocks = unsigned(std::min<int64_t>((n + 255) / 256, 148 * 8));
+  k_validate_graph<<<blocks, 256, 0, s>>>(N, E, rowptr, col, vec);
+  if (cudaGetLastError()) return TPCONV_ERR_CUDA;
+  if (cudaMemcpyFromSymbolAsync(&flag, g_graph_error, sizeof(int), 0, cudaMemcpyDeviceToHost, s)) return TPCONV_ERR_CUDA;
+  if (cudaStreamSynchronize(s)) return TPCONV_ERR_CUDA;
+  return flag ? TPCONV_ERR_GRAPH_INVALID : TPCONV_OK;
+}
+
 int finish(cudaError_t e) {
   if (e != cudaSuccess) return TPCONV_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? TPCONV_OK : TPCONV_ERR_CUDA;
@@ -336,6 +378,8 @@ int tpconv_graph_transpose(const tpconv_plan* plan, int64_t N, int64_t E, const 
   int st = check_ws(plan, TPCONV_OP_TRANSPOSE, N, E, workspace, workspace_bytes, &L);
   if (st) return st;
   cudaStream_t s = S(stream);
+  if ((st = ensure_device())) return st;
+  if ((st = validate_graph(plan, N, E, rowptr, col, nullptr, s))) return st;
   PhaseScope ps(TPCONV_PHASE_TRANSPOSE, s);
   char* ws = static_cast<char*>(workspace);
   int* cnt = reinterpret_cast<int*>(ws + L.off_cursor);
@@ -374,6 +418,7 @@ int tpconv_forward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t*
   if (N == 0) return TPCONV_OK;
   const DevPlan& d = plan->dp;
   cudaStream_t s = S(stream);
+  if ((st = validate_graph(plan, N, E, rowptr, col, edge_vec, s))) return st;
   float* A = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_state);
   float* treg = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_theta);
   const float* thT_hi = nullptr;
@@ -418,6 +463,7 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
   if ((st = ensure_device())) return st;
   const DevPlan& d = plan->dp;
   cudaStream_t s = S(stream);
+  if (N > 0 && (st = validate_graph(plan, N, E, rowptr, col, edge_vec, s))) return st;
   if (dtheta && cudaMemsetAsync(dtheta, 0, plan->theta_numel * 4, s)) return TPCONV_ERR_CUDA;
   if (dx && N > 0 && cudaMemsetAsync(dx, 0, size_t(N) * d.dim_in * 4, s)) return TPCONV_ERR_CUDA;
   if (N == 0) return finish(cudaSuccess);
@@ -487,6 +533,7 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
   if ((st = ensure_device())) return st;
   const DevPlan& d = plan->dp;
   cudaStream_t s = S(stream);
+  if (N > 0 && (st = validate_graph(plan, N, E, rowptr, col, edge_vec, s))) return st;
   const bool has_x1 = gg_x != nullptr, has_v = gg_vec != nullptr, has_t = gg_theta != nullptr;
   if (d_theta && cudaMemsetAsync(d_theta, 0, plan->theta_numel * 4, s)) return TPCONV_ERR_CUDA;
   if (d_x && N > 0 && cudaMemsetAsync(d_x, 0, size_t(N) * d.dim_in * 4, s)) return TPCONV_ERR_CUDA;

@@ -75,7 +75,7 @@ extern "C" {
 /* precision of the node-level Theta contraction (tensor cores) */
 #define TPCONV_GEMM_FP32 0 /* fp32 accuracy: 3xTF32 split on tcgen05      */
 #define TPCONV_GEMM_TF32 1 /* single TF32 pass on tcgen05                 */
-#define TPCONV_GEMM_BF16 2 /* BF16 operands, fp32 accumulate on tcgen05   */
+#define TPCONV_GEMM_BF16 2 /* reserved: plan creation returns UNSUPPORTED */
 #define TPCONV_GEMM_SIMT 3 /* plain fp32 FFMA (reference-precision mode)  */
 
 /* operations, for tpconv_workspace_size */
@@ -92,7 +92,7 @@ typedef struct tpconv_options {
   double radial_p1;      /* Gaussian: r_max; Bessel: unused                   */
   int gemm;              /* TPCONV_GEMM_*                                     */
   size_t workspace_cap;  /* bytes of node-side state per chunk; 0 = no cap    */
-  int validate;          /* 1: check CSR/indices on the device before running */
+  int validate;          /* 1: check the graph on the device first (syncs)    */
 } tpconv_options;
 
 /* Fill *opt with defaults: Bessel (r_cut 5), GEMM_FP32, no cap, no validation. */

@@ -88,3 +88,9 @@ def test_workspace_independent_of_edges_and_capped(T):
         big = T.tpconv_workspace_size(capped, op, 1_222_309, 64_000_000)
         assert big == T.tpconv_workspace_size(capped, op, 500_000, 1_000)
         assert big <= cap + theta_ops + (4 << 20)
+
+
+def test_bf16_mixing_is_reported_unsupported(T):
+    with pytest.raises(T.TPConvError) as e:
+        T.Plan("8x0e+8x1o", 2, "8x0e+8x1o", 4, gemm="bf16")
+    assert e.value.status == 3  # TPCONV_ERR_UNSUPPORTED

@@ -295,3 +295,35 @@ def test_tensor_core_mixing(T, gemm, irr):
     refd = conv.double_backward(prob, rowptr, col, vec, x, th, g, r32(W.normal(x.shape, 62)),
                                 r32(W.normal(vec.shape, 63)), r32(W.normal(th.shape, 64) * 0.05))
     assert rel(dbl["d_g"].cpu().numpy(), refd["d_g"]) < TOL[gemm]
+
+
+def test_validate_mode_rejects_bad_graphs(T):
+    """validate=1: the graph is checked on the device before any stream kernel
+    reads it; a sender index out of range, a broken rowptr or a zero-length edge
+    vector returns TPCONV_ERR_GRAPH_INVALID, a good graph runs normally."""
+    import torch
+    rowptr, col, vec = W.graph_for("tiny", 0)
+    irr = "8x0e+8x1o"
+    plan = T.Plan(irr, 2, irr, 4, radial="gaussian", radial_params=(0.5, 5.0), validate=True)
+    prob = conv.Problem(irr, 2, irr, 4, "gaussian", (0.5, 5.0))
+    N = len(rowptr) - 1
+    x = W.normal((N, prob.dim_in), 71)
+    th = W.theta([(4 * p.c_in * p.c_out, 0.2) for p in prob.paths], 72)
+    xd, thd = dev(x, torch.float32), dev(th, torch.float32)
+    good = T.Graph(dev(rowptr, torch.int32), dev(col, torch.int32), dev(vec, torch.float32))
+    out = T.forward(plan, good, xd, thd)
+    torch.cuda.synchronize()
+    ref = conv.forward(prob, rowptr, col, vec.astype(np.float32).astype(np.float64), x.astype(np.float32),
+                       th.astype(np.float32))
+    assert rel(out.cpu().numpy(), ref) < TOL_FP32
+    bad_col = col.copy()
+    bad_col[5] = N + 3
+    bad_rp = rowptr.copy()
+    bad_rp[7], bad_rp[8] = bad_rp[8], bad_rp[7] - 1
+    bad_vec = vec.copy()
+    bad_vec[11] = 0.0
+    for rp_, col_, vec_ in ((rowptr, bad_col, vec), (bad_rp, col, vec), (rowptr, col, bad_vec)):
+        G = T.Graph(dev(rp_, torch.int32), dev(col_, torch.int32), dev(vec_, torch.float32))
+        with pytest.raises(T.TPConvError) as e:
+            T.forward(plan, G, xd, thd)
+        assert e.value.status == 6  # TPCONV_ERR_GRAPH_INVALID
