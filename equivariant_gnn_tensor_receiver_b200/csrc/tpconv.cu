@@ -137,10 +137,78 @@ bool use_tc(const tpconv_plan* plan) {
 
 // out[r0 : r0+nc] = A . Theta (mode 0) or += (mode 1), per output block.  With
 // thT (Theta^T hi, lo) the tensor-core GEMM runs, else the FFMA GEMM.
+// ---- fork / join of independent launches ----------------------------------
+// The per-block Theta contractions of one call are independent (disjoint
+// output blocks) but each launch alone fills the GPU unevenly (e.g. 32, 96 and
+// 160 tiles of one CTA per SM); issuing them on side streams lets their waves
+// overlap.  Side streams and events are created once per host thread and
+// device; the fork is an event on the caller's stream that each side stream
+// waits for, the join an event per side stream the caller's stream waits for,
+// so the call stays ordered on the caller's stream (and capturable as a fork /
+// join graph once the side resources exist).
+constexpr int kSide = 2;
+struct SideRes {
+  cudaStream_t s[kSide] = {};
+  cudaEvent_t fork = nullptr, join[kSide] = {};
+  bool ok = false;
+};
+SideRes* side_res() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  thread_local SideRes r[kMaxDevices];
+  SideRes& x = r[dev];
+  if (!x.ok) {
+    bool ok = cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < kSide && ok; ++i)
+      ok = cudaStreamCreateWithFlags(&x.s[i], cudaStreamNonBlocking) == cudaSuccess &&
+           cudaEventCreateWithFlags(&x.join[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) return nullptr;  // fall back to the caller's stream
+    x.ok = true;
+  }
+  return &x;
+}
+class ForkJoin {
+ public:
+  explicit ForkJoin(cudaStream_t main) : main_(main), r_(side_res()) {}
+  // stream for the i-th independent piece of work
+  cudaStream_t stream(int i) {
+    const int k = i % (kSide + 1);
+    if (k == 0 || !r_) return main_;
+    if (!forked_) {
+      if (cudaEventRecord(r_->fork, main_) != cudaSuccess) return main_;
+      forked_ = true;
+    }
+    if (!used_[k - 1]) {
+      if (cudaStreamWaitEvent(r_->s[k - 1], r_->fork, 0) != cudaSuccess) return main_;
+      used_[k - 1] = true;
+    }
+    return r_->s[k - 1];
+  }
+  cudaError_t join() {
+    for (int k = 0; k < kSide; ++k) {
+      if (!used_[k]) continue;
+      cudaError_t e = cudaEventRecord(r_->join[k], r_->s[k]);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(main_, r_->join[k], 0);
+      if (e != cudaSuccess) return e;
+      used_[k] = false;
+    }
+    return cudaSuccess;
+  }
+  ~ForkJoin() { join(); }
+
+ private:
+  cudaStream_t main_;
+  SideRes* r_;
+  bool forked_ = false;
+  bool used_[kSide] = {};
+};
+
 cudaError_t node_mix_forward(const tpconv_plan* plan, int r0, int nc, const float* A, const float* theta,
                              const float* thT_hi, const float* thT_lo, float* out, cudaStream_t st, int mode = 0) {
   const DevPlan& d = plan->dp;
+  ForkJoin fj(st);
   for (int i3 = 0; i3 < d.n_out; ++i3) {
+    cudaStream_t si = fj.stream(i3);
     const int n3 = 2 * d.out_l[i3] + 1, cout = d.out_mul[i3];
     const int p0 = first_path_of_out_block(d, i3);
     const int64_t toff = p0 >= 0 ? d.path[p0].theta_off : 0;
@@ -151,17 +219,17 @@ cudaError_t node_mix_forward(const tpconv_plan* plan, int r0, int nc, const floa
       TcOut o{out + size_t(r0) * d.dim_out + d.out_off[i3], n3, d.dim_out, 1, n3};
       const bool split = plan->opt.gemm == TPCONV_GEMM_FP32;
       cudaError_t e = gemm_tc(Ab, Kb, thT_hi + toff, split ? thT_lo + toff : nullptr, Kb, int(M), cout, Kb, o,
-                              mode, split, st);
+                              mode, split, si);
       if (e) return e;
       continue;
     }
     MView a = mrow(F(Ab), Kb);
     MView b = mrow(F(theta + toff), cout);
     MView c = mview(out + size_t(r0) * d.dim_out + d.out_off[i3], n3, d.dim_out, 1, 1, n3, 0);
-    cudaError_t e = gemm_simt(M, cout, Kb, a, b, c, mode, st);
+    cudaError_t e = gemm_simt(M, cout, Kb, a, b, c, mode, si);
     if (e) return e;
   }
-  return cudaSuccess;
+  return fj.join();
 }
 
 // Theta operands of the tensor-core contractions for one Theta (slot 0: Theta,
@@ -216,30 +284,33 @@ cudaError_t prep_tc_theta(const tpconv_plan* plan, const float* theta, float* re
 cudaError_t node_mix_adjoint(const tpconv_plan* plan, int r0, int nc, const float* g, const float* theta,
                              const TcTheta* tc, float* gpack, float* G, cudaStream_t st) {
   const DevPlan& d = plan->dp;
+  ForkJoin fj(st);
   for (int i3 = 0; i3 < d.n_out; ++i3) {
     if (d.Kb[i3] == 0) continue;
+    cudaStream_t si = fj.stream(i3);
+    float* gp = gpack + size_t(nc) * d.out_off[i3];  // this block's slice of the pack region
     const int n3 = 2 * d.out_l[i3] + 1, cout = d.out_mul[i3];
     const int p0 = first_path_of_out_block(d, i3);
     const int64_t toff = d.path[p0].theta_off;
     float* Gb = G + size_t(nc) * d.a_pref[i3];
     const int64_t M = int64_t(nc) * n3;
     cudaError_t e;
-    if (tc && tc->N_hi && gemm_tc_supported(gpack, cout, tc->N_hi + toff, cout, int(M), d.Kb[i3], cout) &&
+    if (tc && tc->N_hi && gemm_tc_supported(gp, cout, tc->N_hi + toff, cout, int(M), d.Kb[i3], cout) &&
         (d.Kb[i3] & 3) == 0) {
-      if ((e = pack_rows(g, d.dim_out, d.out_off[i3], cout, n3, r0, nc, gpack, st))) return e;
+      if ((e = pack_rows(g, d.dim_out, d.out_off[i3], cout, n3, r0, nc, gp, si))) return e;
       TcOut o{Gb, 1, d.Kb[i3], 0, 1};
       const bool split = tc->N_lo != nullptr;
-      if ((e = gemm_tc(gpack, cout, tc->N_hi + toff, split ? tc->N_lo + toff : nullptr, cout, int(M), d.Kb[i3], cout,
-                       o, 0, split, st)))
+      if ((e = gemm_tc(gp, cout, tc->N_hi + toff, split ? tc->N_lo + toff : nullptr, cout, int(M), d.Kb[i3], cout,
+                       o, 0, split, si)))
         return e;
       continue;
     }
     MView a = mview(F(g) + size_t(r0) * d.dim_out + d.out_off[i3], n3, d.dim_out, 1, 1, n3, 0);
     MView b = mview(F(theta) + toff, 1, 1, 0, 1, cout, 0);
     MView c = mrow(Gb, d.Kb[i3]);
-    if ((e = gemm_simt(M, d.Kb[i3], cout, a, b, c, 0, st))) return e;
+    if ((e = gemm_simt(M, d.Kb[i3], cout, a, b, c, 0, si))) return e;
   }
-  return cudaSuccess;
+  return fj.join();
 }
 
 // dx[s0 : s0+nc] += B . Theta (per input block) and dtheta += x^T B (per path)
@@ -247,10 +318,12 @@ cudaError_t node_mix_sender(const tpconv_plan* plan, int s0, int nc, const float
                             const float* theta, const TcTheta* tc, float* dx, float* dtheta, cudaStream_t st) {
   const DevPlan& d = plan->dp;
   cudaError_t e;
+  ForkJoin fj(st);
   if (dx) {
     for (int i1 = 0; i1 < d.n_in; ++i1) {
       const int Kx = d.Kx[i1];
       if (Kx == 0) continue;
+      cudaStream_t si = fj.stream(i1 + 1);  // the Theta gradient runs on the caller's stream
       const int n1 = 2 * d.in_l[i1] + 1, cin = d.in_mul[i1];
       const float* Bb = B + size_t(nc) * d.b_pref[i1];
       const int64_t M = int64_t(nc) * n1;
@@ -260,7 +333,7 @@ cudaError_t node_mix_sender(const tpconv_plan* plan, int s0, int nc, const float
           TcOut o{dx + size_t(s0) * d.dim_in + d.in_off[i1], n1, d.dim_in, 1, n1};
           const bool split = tc->X_lo != nullptr;
           if ((e = gemm_tc(Bb, Kx, tc->X_hi + xo, split ? tc->X_lo + xo : nullptr, Kx, int(M), cin, Kx, o, 1, split,
-                           st)))
+                           si)))
             return e;
           continue;
         }
@@ -271,12 +344,12 @@ cudaError_t node_mix_sender(const tpconv_plan* plan, int s0, int nc, const float
         MView bp = mrow(F(B) + size_t(nc) * d.b_pref[q.i1] + q.kxoff, Kx);
         MView th = mview(F(theta) + q.theta_off, q.c_out, int64_t(q.c_in) * q.c_out, 1, 1, q.c_out, 0);
         MView c = mview(dx + size_t(s0) * d.dim_in + q.in_off, n1, d.dim_in, 1, 1, n1, 0);
-        if ((e = gemm_simt(M, q.c_in, int64_t(d.R) * q.c_out, bp, th, c, 1, st))) return e;
+        if ((e = gemm_simt(M, q.c_in, int64_t(d.R) * q.c_out, bp, th, c, 1, si))) return e;
       }
     }
   }
   if (dtheta && (e = dtheta_accumulate(d, s0, nc, x, B, nullptr, nullptr, dtheta, st))) return e;
-  return cudaSuccess;
+  return fj.join();
 }
 
 // ---- validate mode: the graph is checked on the device before any stream runs ----
