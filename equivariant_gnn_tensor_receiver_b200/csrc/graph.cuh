@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "plan.h"
+
 namespace tpc {
 
 __global__ void k_count_senders(int64_t E, const int* __restrict__ col, int* __restrict__ cnt) {
@@ -94,6 +96,64 @@ __global__ void k_sort_segments(int64_t N, const int* __restrict__ rowptr, const
         else hi = mid;
       }
       s_recv[j0 + rank] = lo;
+    }
+  }
+}
+
+}  // namespace tpc
+
+namespace tpc {
+
+// ---- work lists of the edge streams -----------------------------------------
+// Node i of a chunk owns work item i (its first piece); a node whose CSR segment
+// is longer than `seg` edges owns extra items, one per further piece.  One CTA
+// of 1024 threads writes extra[i] = the first extra item of node i (exclusive
+// scan of the extra counts, in rounds of 1024 with a carry), extra[nc] = their
+// total, and resets the streams' work counter.
+__global__ void __launch_bounds__(1024) k_build_work_list(int nc, const int* __restrict__ ptr, int n0, int seg,
+                                                          int* __restrict__ extra, int* __restrict__ counter) {
+  __shared__ int s[1024];
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base <= nc; base += 1024) {
+    const int i = base + threadIdx.x;
+    int c = 0;
+    if (i < nc) {
+      const int deg = ptr[n0 + i + 1] - ptr[n0 + i];
+      c = deg > seg ? (deg + seg - 1) / seg - 1 : 0;
+    }
+    s[threadIdx.x] = c;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+      const int t = threadIdx.x >= o ? s[threadIdx.x - o] : 0;
+      __syncthreads();
+      s[threadIdx.x] += t;
+      __syncthreads();
+    }
+    if (i <= nc) extra[i] = carry + s[threadIdx.x] - c;
+    __syncthreads();
+    if (threadIdx.x == 1023) carry += s[1023];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *counter = 0;
+}
+
+// zero the state rows of the chunk's multi-piece nodes (their pieces add atomically);
+// recv: A blocks (rows 2l3+1 per node, Kb columns), else B blocks (2l1+1, Kx)
+__global__ void k_zero_heavy_rows(const __grid_constant__ DevPlan pl, int nc, const int* __restrict__ extra,
+                                  bool recv, float* __restrict__ out, float* __restrict__ out0) {
+  for (int i = blockIdx.x; i < nc; i += gridDim.x) {
+    if (extra[i + 1] == extra[i]) continue;
+    const int nb = recv ? pl.n_out : pl.n_in;
+    for (int b = 0; b < nb; ++b) {
+      const int rows = 2 * (recv ? pl.out_l[b] : pl.in_l[b]) + 1;
+      const int width = recv ? pl.Kb[b] : pl.Kx[b];
+      const size_t base = size_t(nc) * (recv ? pl.a_pref[b] : pl.b_pref[b]) + size_t(i) * rows * width;
+      for (int o = threadIdx.x; o < rows * width; o += blockDim.x) {
+        out[base + o] = 0.f;
+        if (out0) out0[base + o] = 0.f;
+      }
     }
   }
 }

@@ -9,18 +9,27 @@
 
 namespace tpc {
 
-inline unsigned wn_grid(int nc) { return unsigned((nc + kWnWarps - 1) / kWnWarps); }
-// path-major grid of the channel-lane streams
-inline unsigned wn_grid_pm(const DevPlan& d, int nc) { return unsigned(d.P) * wn_grid(nc); }
+// path-major grid of the first pieces (channel-lane streams)
+inline unsigned wn_grid_pm(const DevPlan& d, int nc) { return unsigned(d.P) * unsigned((nc + kWnWarps - 1) / kWnWarps); }
+// persistent grid: as many CTAs as fit on the device at once
+template <class K>
+unsigned wn_grid(K kernel, int smem) {
+  int dev = 0, sms = 148, per = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kernel, 32 * kWnWarps, smem) != cudaSuccess || per < 1)
+    per = 1;
+  return unsigned(sms * per);
+}
 
 template <int RM, int LF, int CPL, bool RECV, bool DBL>
 cudaError_t wn_smem(int bytes) {
-  cudaError_t e = cudaFuncSetAttribute(k_wn_stream<RM, LF, CPL, RECV, DBL, false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  cudaError_t e = cudaFuncSetAttribute(k_wn_stream<RM, LF, CPL, RECV, DBL, false, false>, attr, bytes);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_wn_stream<RM, LF, CPL, RECV, DBL, false, true>, attr, bytes);
   if constexpr (DBL) {
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(k_wn_stream<RM, LF, CPL, RECV, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_wn_stream<RM, LF, CPL, RECV, true, true, false>, attr, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_wn_stream<RM, LF, CPL, RECV, true, true, true>, attr, bytes);
   }
   return e;
 }
@@ -37,70 +46,103 @@ cudaError_t wna_smem(int bytes) {
 
 template <int RM, int LF, int CPL>
 cudaError_t launch_wn_fwd(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,
-                          const float* x, float* A, cudaStream_t st) {
+                          const float* x, float* A, const int* extra, int* counter, int seg, cudaStream_t st) {
   if (nc <= 0) return cudaSuccess;
-  k_wn_stream<RM, LF, CPL, true, false, false><<<wn_grid_pm(d, nc), 32 * kWnWarps, d.wn_smem_f, st>>>(
-      d, r0, nc, rowptr, col, nullptr, vec, nullptr, x, nullptr, A, nullptr);
+  auto k = k_wn_stream<RM, LF, CPL, true, false, false, false>;
+  auto kx = k_wn_stream<RM, LF, CPL, true, false, false, true>;
+  k<<<wn_grid_pm(d, nc), 32 * kWnWarps, d.wn_smem_f, st>>>(d, r0, nc, rowptr, col, nullptr, vec, nullptr, x,
+                                                                  nullptr, A, nullptr, extra, counter, seg);
+  kx<<<wn_grid(kx, d.wn_smem_f), 32 * kWnWarps, d.wn_smem_f, st>>>(d, r0, nc, rowptr, col, nullptr, vec, nullptr, x,
+                                                                  nullptr, A, nullptr, extra, counter, seg);
   return cudaGetLastError();
 }
 
 template <int RM, int LF, int CPL>
 cudaError_t launch_wn_send(const DevPlan& d, int s0, int nc, const int* s_rowptr, const int* perm,
-                           const int* s_recv, const float* vec, const float* g, float* B, cudaStream_t st) {
+                           const int* s_recv, const float* vec, const float* g, float* B, const int* extra,
+                           int* counter, int seg, cudaStream_t st) {
   if (nc <= 0) return cudaSuccess;
-  k_wn_stream<RM, LF, CPL, false, false, false><<<wn_grid_pm(d, nc), 32 * kWnWarps, d.wn_smem_s, st>>>(
-      d, s0, nc, s_rowptr, s_recv, perm, vec, nullptr, g, nullptr, B, nullptr);
+  auto k = k_wn_stream<RM, LF, CPL, false, false, false, false>;
+  auto kx = k_wn_stream<RM, LF, CPL, false, false, false, true>;
+  k<<<wn_grid_pm(d, nc), 32 * kWnWarps, d.wn_smem_s, st>>>(d, s0, nc, s_rowptr, s_recv, perm, vec, nullptr, g,
+                                                                  nullptr, B, nullptr, extra, counter, seg);
+  kx<<<wn_grid(kx, d.wn_smem_s), 32 * kWnWarps, d.wn_smem_s, st>>>(d, s0, nc, s_rowptr, s_recv, perm, vec, nullptr, g,
+                                                                  nullptr, B, nullptr, extra, counter, seg);
   return cudaGetLastError();
 }
 
 template <int RM, int LF>
 cudaError_t launch_wn_dbla(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,
                            const float* ggv, const float* x, const float* ggx, float* A1, float* A0,
-                           cudaStream_t st) {
+                           const int* extra, int* counter, int seg, cudaStream_t st) {
   if (nc <= 0) return cudaSuccess;
-  if (A0)
-    k_wn_stream<RM, LF, 1, true, true, true><<<wn_grid_pm(d, nc), 32 * kWnWarps, d.wn_smem_f2, st>>>(
-        d, r0, nc, rowptr, col, nullptr, vec, ggv, x, ggx, A1, A0);
-  else
-    k_wn_stream<RM, LF, 1, true, true, false><<<wn_grid_pm(d, nc), 32 * kWnWarps, d.wn_smem_f2, st>>>(
-        d, r0, nc, rowptr, col, nullptr, vec, ggv, x, ggx, A1, nullptr);
+  if (A0) {
+    auto k = k_wn_stream<RM, LF, 1, true, true, true, false>;
+    auto kx = k_wn_stream<RM, LF, 1, true, true, true, true>;
+    k<<<wn_grid_pm(d, nc), 32 * kWnWarps, d.wn_smem_f2, st>>>(d, r0, nc, rowptr, col, nullptr, vec, ggv, x,
+                                                                      ggx, A1, A0, extra, counter, seg);
+    kx<<<wn_grid(kx, d.wn_smem_f2), 32 * kWnWarps, d.wn_smem_f2, st>>>(d, r0, nc, rowptr, col, nullptr, vec, ggv, x,
+                                                                      ggx, A1, A0, extra, counter, seg);
+  } else {
+    auto k = k_wn_stream<RM, LF, 1, true, true, false, false>;
+    auto kx = k_wn_stream<RM, LF, 1, true, true, false, true>;
+    k<<<wn_grid_pm(d, nc), 32 * kWnWarps, d.wn_smem_f2, st>>>(d, r0, nc, rowptr, col, nullptr, vec, ggv, x,
+                                                                      ggx, A1, nullptr, extra, counter, seg);
+    kx<<<wn_grid(kx, d.wn_smem_f2), 32 * kWnWarps, d.wn_smem_f2, st>>>(d, r0, nc, rowptr, col, nullptr, vec, ggv, x,
+                                                                      ggx, A1, nullptr, extra, counter, seg);
+  }
   return cudaGetLastError();
 }
 
 template <int RM, int LF>
 cudaError_t launch_wn_dbls(const DevPlan& d, int s0, int nc, const int* s_rowptr, const int* perm,
                            const int* s_recv, const float* vec, const float* ggv, const float* g, float* B1,
-                           float* B0, cudaStream_t st) {
+                           float* B0, const int* extra, int* counter, int seg, cudaStream_t st) {
   if (nc <= 0) return cudaSuccess;
-  if (B0)
-    k_wn_stream<RM, LF, 1, false, true, true><<<wn_grid_pm(d, nc), 32 * kWnWarps, d.wn_smem_s2, st>>>(
-        d, s0, nc, s_rowptr, s_recv, perm, vec, ggv, g, nullptr, B1, B0);
-  else
-    k_wn_stream<RM, LF, 1, false, true, false><<<wn_grid_pm(d, nc), 32 * kWnWarps, d.wn_smem_s2, st>>>(
-        d, s0, nc, s_rowptr, s_recv, perm, vec, ggv, g, nullptr, B1, nullptr);
+  if (B0) {
+    auto k = k_wn_stream<RM, LF, 1, false, true, true, false>;
+    auto kx = k_wn_stream<RM, LF, 1, false, true, true, true>;
+    k<<<wn_grid_pm(d, nc), 32 * kWnWarps, d.wn_smem_s2, st>>>(d, s0, nc, s_rowptr, s_recv, perm, vec, ggv, g,
+                                                                      nullptr, B1, B0, extra, counter, seg);
+    kx<<<wn_grid(kx, d.wn_smem_s2), 32 * kWnWarps, d.wn_smem_s2, st>>>(d, s0, nc, s_rowptr, s_recv, perm, vec, ggv, g,
+                                                                      nullptr, B1, B0, extra, counter, seg);
+  } else {
+    auto k = k_wn_stream<RM, LF, 1, false, true, false, false>;
+    auto kx = k_wn_stream<RM, LF, 1, false, true, false, true>;
+    k<<<wn_grid_pm(d, nc), 32 * kWnWarps, d.wn_smem_s2, st>>>(d, s0, nc, s_rowptr, s_recv, perm, vec, ggv, g,
+                                                                      nullptr, B1, nullptr, extra, counter, seg);
+    kx<<<wn_grid(kx, d.wn_smem_s2), 32 * kWnWarps, d.wn_smem_s2, st>>>(d, s0, nc, s_rowptr, s_recv, perm, vec, ggv, g,
+                                                                      nullptr, B1, nullptr, extra, counter, seg);
+  }
   return cudaGetLastError();
 }
 
 template <int RM, int LF>
 cudaError_t launch_wn_adj(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,
-                          const float* x, const float* G, float* dvec, float* dY, float* db, cudaStream_t st) {
+                          const float* x, const float* G, float* dvec, float* dY, float* db, const int* extra,
+                          int* counter, cudaStream_t st) {
   if (nc <= 0) return cudaSuccess;
-  k_wn_adj<RM, LF, false, false><<<wn_grid(nc), 32 * kWnWarps, d.wn_smem_adj, st>>>(
-      d, r0, nc, rowptr, col, vec, nullptr, x, nullptr, G, nullptr, dvec, dY, db);
+  auto k = k_wn_adj<RM, LF, false, false>;
+  k<<<wn_grid(k, d.wn_smem_adj), 32 * kWnWarps, d.wn_smem_adj, st>>>(d, r0, nc, rowptr, col, vec, nullptr, x, nullptr,
+                                                                      G, nullptr, dvec, dY, db, extra, counter);
   return cudaGetLastError();
 }
 
 template <int RM, int LF>
 cudaError_t launch_wn_dadj(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,
                            const float* ggv, const float* x, const float* ggx, const float* G, const float* Gt,
-                           float* dvec, cudaStream_t st) {
+                           float* dvec, const int* extra, int* counter, cudaStream_t st) {
   if (nc <= 0) return cudaSuccess;
-  if (Gt)
-    k_wn_adj<RM, LF, true, true><<<wn_grid(nc), 32 * kWnWarps, d.wn_smem_dadj, st>>>(
-        d, r0, nc, rowptr, col, vec, ggv, x, ggx, G, Gt, dvec, nullptr, nullptr);
-  else
-    k_wn_adj<RM, LF, true, false><<<wn_grid(nc), 32 * kWnWarps, d.wn_smem_dadj, st>>>(
-        d, r0, nc, rowptr, col, vec, ggv, x, ggx, G, nullptr, dvec, nullptr, nullptr);
+  if (Gt) {
+    auto k = k_wn_adj<RM, LF, true, true>;
+    k<<<wn_grid(k, d.wn_smem_dadj), 32 * kWnWarps, d.wn_smem_dadj, st>>>(d, r0, nc, rowptr, col, vec, ggv, x, ggx, G,
+                                                                          Gt, dvec, nullptr, nullptr, extra, counter);
+  } else {
+    auto k = k_wn_adj<RM, LF, true, false>;
+    k<<<wn_grid(k, d.wn_smem_dadj), 32 * kWnWarps, d.wn_smem_dadj, st>>>(d, r0, nc, rowptr, col, vec, ggv, x, ggx, G,
+                                                                          nullptr, dvec, nullptr, nullptr, extra,
+                                                                          counter);
+  }
   return cudaGetLastError();
 }
 

@@ -37,24 +37,27 @@ cudaError_t launch_dbl_r_rm(const DevPlan& d, int r0, int nc, const int* rowptr,
 // the number of channels per lane of the channel-lane forms.
 template <int RM, int LF, int CPL>
 cudaError_t launch_wn_fwd(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,
-                          const float* x, float* A, cudaStream_t st);
+                          const float* x, float* A, const int* extra, int* counter, int seg, cudaStream_t st);
 template <int RM, int LF, int CPL>
 cudaError_t launch_wn_send(const DevPlan& d, int s0, int nc, const int* s_rowptr, const int* perm,
-                           const int* s_recv, const float* vec, const float* g, float* B, cudaStream_t st);
+                           const int* s_recv, const float* vec, const float* g, float* B, const int* extra,
+                           int* counter, int seg, cudaStream_t st);
 template <int RM, int LF>
 cudaError_t launch_wn_dbla(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,
-                           const float* ggv, const float* x, const float* ggx, float* A1, float* A0, cudaStream_t st);
+                           const float* ggv, const float* x, const float* ggx, float* A1, float* A0,
+                           const int* extra, int* counter, int seg, cudaStream_t st);
 template <int RM, int LF>
 cudaError_t launch_wn_dbls(const DevPlan& d, int s0, int nc, const int* s_rowptr, const int* perm,
                            const int* s_recv, const float* vec, const float* ggv, const float* g, float* B1,
-                           float* B0, cudaStream_t st);
+                           float* B0, const int* extra, int* counter, int seg, cudaStream_t st);
 template <int RM, int LF>
 cudaError_t launch_wn_adj(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,
-                          const float* x, const float* G, float* dvec, float* dY, float* db, cudaStream_t st);
+                          const float* x, const float* G, float* dvec, float* dY, float* db, const int* extra,
+                          int* counter, cudaStream_t st);
 template <int RM, int LF>
 cudaError_t launch_wn_dadj(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,
                            const float* ggv, const float* x, const float* ggx, const float* G, const float* Gt,
-                           float* dvec, cudaStream_t st);
+                           float* dvec, const int* extra, int* counter, cudaStream_t st);
 
 // instantiation of a warp-per-node launcher for the plan's (rm, wn_lf[, wn_cpl])
 #define TPC_WN_CALL(d, fn, ...)                                                                \

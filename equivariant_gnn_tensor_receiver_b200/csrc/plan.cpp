@@ -491,6 +491,9 @@ int tpc::ws_layout(const tpconv_plan& p, int op, int64_t N, int64_t E, WsLayout*
   L->off_pack = off;
   L->pack_bytes = align256(size_t(Nc) * size_t(p.dp.dim_out) * 4);
   off = align256(off + L->pack_bytes);
+  L->off_lists = off;
+  L->list_ints = work_list_ints(Nc);
+  off = align256(off + size_t(kWorkLists) * L->list_ints * 4);
   L->total = off;
   return TPCONV_OK;
 }

@@ -89,7 +89,7 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
                                              const int* __restrict__ perm, const float* __restrict__ vec,
                                              const float* __restrict__ ggv, const float* __restrict__ src,
                                              const float* __restrict__ src1, float* __restrict__ out,
-                                             float* __restrict__ out0) {
+                                             float* __restrict__ out0, bool split) {
   using TR = Tri<L1, L2, L3>;
   constexpr int N2 = TR::N2, NMZ = TR::NMZ, NMP = (NMZ + 3) & ~3;
   constexpr int NI = RECV ? TR::N1 : TR::N3;  // staged floats per channel
@@ -272,46 +272,83 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
           for (int i = 0; i < NO; ++i) {
             const float2 v = acc[((part * CPL + h) * NK2 + kp) * NO + i];
             float* d = dst + base + size_t(i) * Kq + ch;
-            if (2 * kp < pl.R) d[size_t(2 * kp) * c] = v.x;
-            if (2 * kp + 1 < pl.R) d[size_t(2 * kp + 1) * c] = v.y;
+            if (split) {  // one piece of a long segment: add into the zeroed rows
+              if (2 * kp < pl.R) atomicAdd(d + size_t(2 * kp) * c, v.x);
+              if (2 * kp + 1 < pl.R) atomicAdd(d + size_t(2 * kp + 1) * c, v.y);
+            } else {
+              if (2 * kp < pl.R) d[size_t(2 * kp) * c] = v.x;
+              if (2 * kp + 1 < pl.R) d[size_t(2 * kp + 1) * c] = v.y;
+            }
           }
       }
     }
   }
 }
 
-// grid: P * ceil(nc / kWnWarps) CTAs of kWnWarps warps, path-major: CTA b runs
-// path b / nblk for nodes n0 + (b % nblk) * kWnWarps + warp.  CTAs are dispatched
-// roughly in index order, so the CTAs resident at any time run one or two path
-// bodies and share their instructions in the instruction caches.
+// Two launches per call.  First (EXTRA = false): a path-major grid of
+// P * ceil(nc / kWnWarps) CTAs, CTA b running path b / nblk for nodes
+// (b % nblk) * kWnWarps + warp; each warp takes its node's whole segment, or the
+// first `seg` edges of a longer one.  CTAs are dispatched roughly in index
+// order, so the resident warps share one or two path bodies in the instruction
+// caches.  Second (EXTRA = true): a persistent grid whose warps claim the
+// further pieces of long segments, path-major, from *counter (list `extra`,
+// see graph.cuh); it ends at once when no segment is split.  A node with one
+// piece stores its state rows; a split node's pieces add into rows zeroed
+// beforehand.
 // RECV: ptr = rowptr, nbr = col (edge id = CSR position); else ptr = s_rowptr,
 // nbr = s_recv, perm = sender-sorted position -> edge id.
-template <int RM, int LF, int CPL, bool RECV, bool DBL, bool P1>
+template <int RM, int LF, int CPL, bool RECV, bool DBL, bool P1, bool EXTRA>
 __global__ void __launch_bounds__(32 * kWnWarps, DBL && RECV ? 3 : 4)
     k_wn_stream(const __grid_constant__ DevPlan pl, int n0, int nc, const int* __restrict__ ptr,
                 const int* __restrict__ nbr, const int* __restrict__ perm, const float* __restrict__ vec,
                 const float* __restrict__ ggv, const float* __restrict__ src, const float* __restrict__ src1,
-                float* __restrict__ out, float* __restrict__ out0) {
+                float* __restrict__ out, float* __restrict__ out0, const int* __restrict__ extra,
+                int* __restrict__ counter, int seg) {
   extern __shared__ __align__(16) float sm[];
-  const int warp = threadIdx.x >> 5;
-  const int nblk = (nc + kWnWarps - 1) / kWnWarps;
-  const int p = blockIdx.x / nblk;
-  const int nl = (blockIdx.x - p * nblk) * kWnWarps + warp;
-  if (nl >= nc) return;
+  const int warp = threadIdx.x >> 5, lane = lane_id();
   const WnLay L = wn_layout_of(RM, CPL, RECV ? pl.n1max : pl.n3max, pl.nmz_max, DBL, DBL && RECV);
   float* ws = sm + warp * L.total;
-  const int a0 = ptr[n0 + nl], a1 = ptr[n0 + nl + 1];
-  const DevPath& q = pl.path[p];
-  switch (triple_id(q.l1, q.l2, q.l3)) {
+  int claim = 0, ne = 0, total = 0;
+  if constexpr (EXTRA) {
+    ne = extra[nc];
+    total = pl.P * ne;
+    if (total == 0) return;
+    // the next piece is claimed while the current one runs (hides the atomic's latency)
+    claim = lane == 0 ? atomicAdd(counter, 1) : 0;
+  }
+  for (;;) {  // first launch: one pass; second launch: the claimed pieces
+    int p, nl, k;
+    if constexpr (!EXTRA) {
+      const int nblk = (nc + kWnWarps - 1) / kWnWarps;
+      p = blockIdx.x / nblk;
+      nl = (blockIdx.x - p * nblk) * kWnWarps + warp;
+      k = 0;
+      if (nl >= nc) break;
+    } else {
+      const int g = __shfl_sync(0xffffffffu, claim, 0);
+      if (g >= total) break;
+      if (lane == 0) claim = atomicAdd(counter, 1);
+      p = g / ne;
+      const int u = g - p * ne;
+      nl = extra_owner(extra, nc, u);
+      k = 1 + (u - extra[nl]);
+    }
+    const int s0 = ptr[n0 + nl], s1 = ptr[n0 + nl + 1];
+    const int a0 = s0 + k * seg, a1 = min(s1, a0 + seg);
+    const bool split = s1 - s0 > seg;
+    const DevPath& q = pl.path[p];
+    switch (triple_id(q.l1, q.l2, q.l3)) {
 #define TPC_CASE(a, b, c)                                                                                        \
   case triple_id(a, b, c):                                                                                       \
     if constexpr (a <= LF && c <= LF)                                                                            \
       wn_chan_path<a, b, c, RM, CPL, RECV, DBL, P1>(pl, q, L, ws, nl, nc, a0, a1, nbr, perm, vec, ggv, src, src1, \
-                                                    out, out0);                                                  \
+                                                    out, out0, split);                                           \
     break;
-    TPC_FOR_EACH_TRIPLE(TPC_CASE)
+      TPC_FOR_EACH_TRIPLE(TPC_CASE)
 #undef TPC_CASE
-    default: break;
+      default: break;
+    }
+    if constexpr (!EXTRA) break;
   }
 }
 

@@ -291,11 +291,13 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
   }
 }
 
-// grid: ceil(nc / kWnWarps) CTAs of kWnWarps warps; warp = receiver r0 + rl.
-// The warps of a CTA step through the paths together (one barrier per path), so
-// that the resident warps of an SM share one or two path bodies in the
-// instruction caches; every warp runs the CTA's largest batch count, the ones
-// with fewer batches (or no node) joining the barriers without work.
+// Persistent grid of kWnWarps-warp CTAs.  A CTA takes kWnWarps work items per
+// round from *counter; an item is one batch of up to 32 edges of a receiver:
+// item t < nc is receiver t's first batch, item t >= nc a further batch (list
+// `extra`, built with seg = 32).  The warps of a CTA step through the paths
+// together (one barrier per path), so the resident warps of an SM share one or
+// two path bodies in the instruction caches, and every warp of a round has at
+// most one batch, so the rounds stay balanced whatever the degrees.
 // First order writes dvec (and, when given, dY [E][n_sh], db [E][R]); second
 // order writes dvec.  x1 / ggv may be null (their terms vanish); Gt is used
 // exactly when GT.
@@ -305,25 +307,38 @@ __global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
              const int* __restrict__ col, const float* __restrict__ vec, const float* __restrict__ ggv,
              const float* __restrict__ x, const float* __restrict__ x1, const float* __restrict__ G,
              const float* __restrict__ Gt, float* __restrict__ dvec, float* __restrict__ dYout,
-             float* __restrict__ dbout) {
+             float* __restrict__ dbout, const int* __restrict__ extra, int* __restrict__ counter) {
   extern __shared__ __align__(16) float sm[];
   const int warp = threadIdx.x >> 5, lane = lane_id();
-  const int rl = blockIdx.x * kWnWarps + warp;
-  const bool has_node = rl < nc;
   const WnaLay L = wna_layout_of(RM, pl.n3max, pl.n1max, DBL);
-  int& s_nbat = *reinterpret_cast<int*>(sm + kWnWarps * L.total);  // CTA batch count
   float* ws = sm + warp * L.total;
+  int& s_base = *reinterpret_cast<int*>(sm + kWnWarps * L.total);  // this round's first item
   // staged buffers read where nothing was staged must hold zeros
   for (int i = lane; i < L.Geo; i += 32) ws[i] = 0.f;
-  const int e0 = has_node ? rowptr[r0 + rl] : 0, e1 = has_node ? rowptr[r0 + rl + 1] : 0;
-  if (threadIdx.x == 0) s_nbat = 0;
-  __syncthreads();
-  if (lane == 0 && e1 > e0) atomicMax(&s_nbat, (e1 - e0 + 31) / 32);
-  __syncthreads();
-  const int nbat = s_nbat;
-  for (int bi = 0; bi < nbat; ++bi) {
-    const int eb = e0 + 32 * bi;
-    const int nb = max(0, min(32, e1 - eb));
+  const int total = nc + extra[nc];
+  // the next round is claimed while the current one runs (hides the atomic's latency)
+  int claim = threadIdx.x == 0 ? atomicAdd(counter, kWnWarps) : 0;
+  for (;;) {
+    __syncthreads();  // every warp has read the previous round's s_base
+    if (threadIdx.x == 0) {
+      s_base = claim;
+      claim = atomicAdd(counter, kWnWarps);
+    }
+    __syncthreads();
+    const int t = s_base + warp;
+    if (s_base >= total) break;  // uniform over the CTA
+    int rl = -1, eb = 0, nb = 0;
+    if (t < total) {
+      rl = t;
+      int k = 0;
+      if (t >= nc) {
+        rl = extra_owner(extra, nc, t - nc);
+        k = 1 + (t - nc - extra[rl]);
+      }
+      const int e0 = rowptr[r0 + rl], e1 = rowptr[r0 + rl + 1];
+      eb = e0 + kBatchEdges * k;
+      nb = max(0, min(kBatchEdges, e1 - eb));
+    }
     const bool valid = lane < nb;
     const int e = eb + lane;
     int myrow = 0;
@@ -373,7 +388,7 @@ __global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
 #define TPC_CASE(a, b, c)                                                                                 \
   case triple_id(a, b, c):                                                                                \
     if constexpr (a <= LF && c <= LF)                                                                     \
-      wna_path<a, b, c, RM, DBL, GT>(pl, q, L, ws, rl, nc, nb, myrow, x, x1, G, Gt, db2, hb2);                  \
+      wna_path<a, b, c, RM, DBL, GT>(pl, q, L, ws, rl, nc, nb, myrow, x, x1, G, Gt, db2, hb2);              \
     break;
           TPC_FOR_EACH_TRIPLE(TPC_CASE)
 #undef TPC_CASE

@@ -24,6 +24,7 @@
 #include "graph.cuh"
 #include "launchers.h"
 #include "plan.h"
+#include "wn_layout.h"
 #include "workspace.h"
 
 using namespace tpc;
@@ -352,6 +353,34 @@ cudaError_t node_mix_sender(const tpconv_plan* plan, int s0, int nc, const float
   return fj.join();
 }
 
+// ---- work lists of the edge streams (graph.cuh) ------------------------------
+struct WorkList {
+  int* counter;
+  int* extra;  // exclusive scan of the nodes' extra items; extra[nc] = their total
+};
+WorkList work_list(const WsLayout& L, void* ws, int which, int64_t chunk_nodes) {
+  int* base = reinterpret_cast<int*>(static_cast<char*>(ws) + L.off_lists) + size_t(which) * L.list_ints;
+  return WorkList{base, base + 32 + work_list_pad(chunk_nodes)};
+}
+// pieces of at most seg edges for the nodes n0 .. n0+nc-1 of ptr; resets the counter
+cudaError_t build_work_list(const WorkList& wl, const WsLayout& L, const int* ptr, int n0, int nc, int seg,
+                            cudaStream_t s) {
+  (void)L;
+  k_build_work_list<<<1, 1024, 0, s>>>(nc, ptr, n0, seg, wl.extra, wl.counter);
+  return cudaGetLastError();
+}
+// piece length of the channel-lane streams: nodes far above the mean degree split
+int piece_edges(int64_t N, int64_t E) {
+  const int64_t mean = N > 0 ? (E + N - 1) / N : 0;
+  return int(std::max<int64_t>(256, 4 * mean));
+}
+// zero the state rows of the chunk's split nodes (their pieces add atomically)
+cudaError_t zero_split_rows(const DevPlan& d, int nc, const WorkList& wl, bool recv, float* out, float* out0,
+                            cudaStream_t s) {
+  k_zero_heavy_rows<<<unsigned(std::max(1, std::min(nc, 1184))), 128, 0, s>>>(d, nc, wl.extra, recv, out, out0);
+  return cudaGetLastError();
+}
+
 // ---- validate mode: the graph is checked on the device before any stream runs ----
 __device__ int g_graph_error;
 
@@ -508,8 +537,14 @@ int tpconv_forward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t*
     const int nc = int(std::min<int64_t>(L.chunk_nodes, N - r0));
     {
       PhaseScope ps(TPCONV_PHASE_FWD_EDGE, s);
-      if (TPC_WN_CALL_CPL(d, launch_wn_fwd, d, int(r0), nc, rowptr, col, edge_vec, x, A, s)) return TPCONV_ERR_CUDA;
-      note(TPCONV_PHASE_FWD_EDGE, 1);
+      const WorkList wl = work_list(L, workspace, 0, L.chunk_nodes);
+      const int seg = piece_edges(N, E);
+      if (build_work_list(wl, L, rowptr, int(r0), nc, seg, s) || zero_split_rows(d, nc, wl, true, A, nullptr, s))
+        return TPCONV_ERR_CUDA;
+      if (TPC_WN_CALL_CPL(d, launch_wn_fwd, d, int(r0), nc, rowptr, col, edge_vec, x, A, wl.extra, wl.counter, seg,
+                          s))
+        return TPCONV_ERR_CUDA;
+      note(TPCONV_PHASE_FWD_EDGE, 4);  // list, zeroed split rows, two stream launches
     }
     {
       PhaseScope ps(TPCONV_PHASE_FWD_NODE, s);
@@ -561,13 +596,16 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
       }
       {
         PhaseScope ps(TPCONV_PHASE_BWD_EDGE_R, s);
-        cudaError_t e = d.wn_ok && aligned16(x)
+        const bool wn = d.wn_ok && aligned16(x);
+        const WorkList wl = work_list(L, workspace, 1, L.chunk_nodes);
+        if (wn && build_work_list(wl, L, rowptr, int(r0), nc, kBatchEdges, s)) return TPCONV_ERR_CUDA;
+        cudaError_t e = wn
                             ? TPC_WN_CALL(d, launch_wn_adj, d, int(r0), nc, rowptr, col, edge_vec, x, S_, dvec, dY, db,
-                                          s)
+                                          wl.extra, wl.counter, s)
                             : TPC_RM_CALL(d.rm, launch_radj_rm, d, int(r0), nc, rowptr, col, edge_vec, x, S_, dvec,
                                           dY, db, s);
         if (e) return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_BWD_EDGE_R, 1);
+        note(TPCONV_PHASE_BWD_EDGE_R, wn ? 2 : 1);
       }
     }
   }
@@ -576,8 +614,15 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
       const int nc = int(std::min<int64_t>(L.chunk_nodes, N - s0));
       {
         PhaseScope ps(TPCONV_PHASE_BWD_EDGE_S, s);
-        if (TPC_WN_CALL_CPL(d, launch_wn_send, d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, g, S_, s)) return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_BWD_EDGE_S, 1);
+        const WorkList wl = work_list(L, workspace, 2, L.chunk_nodes);
+        const int seg = piece_edges(N, E);
+        if (build_work_list(wl, L, s_rowptr, int(s0), nc, seg, s) ||
+            zero_split_rows(d, nc, wl, false, S_, nullptr, s))
+          return TPCONV_ERR_CUDA;
+        if (TPC_WN_CALL_CPL(d, launch_wn_send, d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, g, S_, wl.extra,
+                            wl.counter, seg, s))
+          return TPCONV_ERR_CUDA;
+        note(TPCONV_PHASE_BWD_EDGE_S, 4);  // list, zeroed split rows, two stream launches
       }
       {
         PhaseScope ps(TPCONV_PHASE_BWD_NODE_X, s);
@@ -640,10 +685,15 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
       const int nc = int(std::min<int64_t>(Nc, N - r0));
       {
         PhaseScope ps(TPCONV_PHASE_DBL_EDGE_A, s);
-        if (TPC_WN_CALL(d, launch_wn_dbla, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, A1,
-                        has_t ? A0 : nullptr, s))
+        const WorkList wl = work_list(L, workspace, 0, L.chunk_nodes);
+        const int seg = piece_edges(N, E);
+        if (build_work_list(wl, L, rowptr, int(r0), nc, seg, s) ||
+            zero_split_rows(d, nc, wl, true, A1, has_t ? A0 : nullptr, s))
           return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_DBL_EDGE_A, 1);
+        if (TPC_WN_CALL(d, launch_wn_dbla, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, A1,
+                        has_t ? A0 : nullptr, wl.extra, wl.counter, seg, s))
+          return TPCONV_ERR_CUDA;
+        note(TPCONV_PHASE_DBL_EDGE_A, 4);  // list, zeroed split rows, two stream launches
       }
       PhaseScope ps(TPCONV_PHASE_DBL_NODE_A, s);
       if (node_mix_forward(plan, int(r0), nc, A1, theta, t_hi, t_lo, d_g, s, 0)) return TPCONV_ERR_CUDA;
@@ -670,13 +720,16 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
         }
       }
       PhaseScope ps(TPCONV_PHASE_DBL_EDGE_R, s);
-      cudaError_t e = d.wn_ok && aligned16(x) && aligned16(gg_x)
+      const bool wn = d.wn_ok && aligned16(x) && aligned16(gg_x);
+      const WorkList wl = work_list(L, workspace, 1, L.chunk_nodes);
+      if (wn && build_work_list(wl, L, rowptr, int(r0), nc, kBatchEdges, s)) return TPCONV_ERR_CUDA;
+      cudaError_t e = wn
                           ? TPC_WN_CALL(d, launch_wn_dadj, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, G,
-                                        has_t ? Gt : nullptr, d_vec, s)
+                                        has_t ? Gt : nullptr, d_vec, wl.extra, wl.counter, s)
                           : TPC_RM_CALL(d.rm, launch_dbl_r_rm, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x,
                                         gg_x, G, has_t ? Gt : nullptr, d_vec, s);
       if (e) return TPCONV_ERR_CUDA;
-      note(TPCONV_PHASE_DBL_EDGE_R, 1);
+      note(TPCONV_PHASE_DBL_EDGE_R, wn ? 2 : 1);
     }
   }
   // d_x = B1 . Theta + B0 . gg_theta ;  d_theta = x^T B1 + gg_x^T B0
@@ -687,10 +740,15 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
       const int nc = int(std::min<int64_t>(Nc, N - s0));
       {
         PhaseScope ps(TPCONV_PHASE_DBL_EDGE_S, s);
-        if (TPC_WN_CALL(d, launch_wn_dbls, d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, gg_vec, g, B1,
-                        (has_x1 || has_t) ? B0 : nullptr, s))
+        float* B0u = (has_x1 || has_t) ? B0 : nullptr;
+        const WorkList wl = work_list(L, workspace, 2, L.chunk_nodes);
+        const int seg = piece_edges(N, E);
+        if (build_work_list(wl, L, s_rowptr, int(s0), nc, seg, s) || zero_split_rows(d, nc, wl, false, B1, B0u, s))
           return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_DBL_EDGE_S, 1);
+        if (TPC_WN_CALL(d, launch_wn_dbls, d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, gg_vec, g, B1, B0u,
+                        wl.extra, wl.counter, seg, s))
+          return TPCONV_ERR_CUDA;
+        note(TPCONV_PHASE_DBL_EDGE_S, 4);  // list, zeroed split rows, two stream launches
       }
       PhaseScope ps(TPCONV_PHASE_DBL_NODE_X, s);
       float* dx1 = has_v ? d_x : nullptr;

@@ -1,4 +1,4 @@
 // Warp-per-node stream (sender form, second order), radial width 4, feature degrees <= 3.
 #include "launch_wn.cuh"
 
-TPC_WN_TU(wn_dbls_r4_l3, dbls, 4, 3, false, true, const DevPlan&, int, int, const int*, const int*, const int*, const float*, const float*, const float*, float*, float*, cudaStream_t)
+TPC_WN_TU(wn_dbls_r4_l3, dbls, 4, 3, false, true, const DevPlan&, int, int, const int*, const int*, const int*, const float*, const float*, const float*, float*, float*, const int*, int*, int, cudaStream_t)

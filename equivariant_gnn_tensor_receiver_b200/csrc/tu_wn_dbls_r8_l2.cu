@@ -1,4 +1,4 @@
 // Warp-per-node stream (sender form, second order), radial width 8, feature degrees <= 2.
 #include "launch_wn.cuh"
 
-TPC_WN_TU(wn_dbls_r8_l2, dbls, 8, 2, false, true, const DevPlan&, int, int, const int*, const int*, const int*, const float*, const float*, const float*, float*, float*, cudaStream_t)
+TPC_WN_TU(wn_dbls_r8_l2, dbls, 8, 2, false, true, const DevPlan&, int, int, const int*, const int*, const int*, const float*, const float*, const float*, float*, float*, const int*, int*, int, cudaStream_t)

@@ -1,4 +1,4 @@
 // Warp-per-node stream (receiver form, first order), radial width 8, feature degrees <= 3, 1 channel(s) per lane.
 #include "launch_wn.cuh"
 
-TPC_WN_TU_CPL(wn_fwd_r8_l3_c1, fwd, 8, 3, 1, true, false, const DevPlan&, int, int, const int*, const int*, const float*, const float*, float*, cudaStream_t)
+TPC_WN_TU_CPL(wn_fwd_r8_l3_c1, fwd, 8, 3, 1, true, false, const DevPlan&, int, int, const int*, const int*, const float*, const float*, float*, const int*, int*, int, cudaStream_t)

@@ -83,4 +83,22 @@ TPC_HD inline int wna_smem_bytes(int RM, int n3max, int n1max, bool dbl) {
   return kWnWarps * wna_layout_of(RM, n3max, n1max, dbl).total * 4 + 16;
 }
 
+// ---- work items of the streams (lists built in graph.cuh) ----
+// Item t < nc is node t's first piece; item t >= nc is extra piece t - nc.
+constexpr int kBatchEdges = 32;  // edges per adjoint work item (lane = edge)
+
+#if defined(__CUDACC__)
+// item t >= nc: the extra piece u = t - nc belongs to the node i with extra[i] <= u < extra[i+1]
+__device__ __forceinline__ int extra_owner(const int* __restrict__ extra, int nc, int u) {
+  int lo = 0, hi = nc;  // extra[lo] <= u < extra[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (extra[mid] <= u) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
+
+#endif
+
 }  // namespace tpc

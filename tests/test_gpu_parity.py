@@ -114,6 +114,43 @@ def test_edge_cases_empty_and_hub(T):
             assert rel(bw[k], rb[k]) < TOL_FP32, (cap, k)
 
 
+def test_power_law_hubs_split_into_pieces(T):
+    """Heavy-tailed degrees: three hub receivers (1500, 900, 600 in-edges) and
+    two hub senders (1200 out-edges each) over a sparse background.  Segments
+    longer than max(256, 4 x mean degree) edges run as several pieces that add
+    into zeroed state rows, and the receivers' batches are spread over warps;
+    forward, backward and double backward against the oracle."""
+    import torch
+    g = W.rng(17)
+    N = 400
+    bg_r, bg_s = g.integers(0, N, size=3200), g.integers(0, N, size=3200)
+    recv = np.concatenate([np.full(1500, 11), np.full(900, 203), np.full(600, 390), bg_r,
+                           g.integers(0, N, size=2400)])
+    send = np.concatenate([g.integers(0, N, size=3000), bg_s, np.full(1200, 77), np.full(1200, 298)])
+    E = len(recv)
+    dvec = g.normal(size=(E, 3))
+    vec = dvec / np.linalg.norm(dvec, axis=1, keepdims=True) * g.uniform(0.6, 4.8, size=(E, 1))
+    graph = W._to_csr(N, send, recv, vec)
+    irr_in, irr_out = "8x0e+8x1o+4x2e", "8x0e+4x1o+8x2e"
+    plan, prob, G, inp = make(T, irr_in, 2, irr_out, 8, "bessel", (5.0,), graph, seed=23)
+    rowptr, col, vec32, x, th, gg = inp
+    assert np.diff(rowptr).max() > 4 * 256 and np.bincount(col).max() >= 1200
+    out, bw = run_fwd_bwd(T, plan, G, inp)
+    assert rel(out, conv.forward(prob, rowptr, col, vec32, x, th)) < TOL_FP32
+    rb = conv.backward(prob, rowptr, col, vec32, x, th, gg)
+    for k in ("dx", "dtheta", "dvec"):
+        assert rel(bw[k], rb[k]) < TOL_FP32, k
+    r32 = lambda a: a.astype(np.float32).astype(np.float64)
+    ggx, ggv = r32(W.normal(x.shape, 24)), r32(W.normal(vec32.shape, 25))
+    ggt = r32(W.normal(th.shape, 26) * 0.05)
+    o2 = T.double_backward(plan, G, dev(x, torch.float32), dev(th, torch.float32), dev(gg, torch.float32),
+                           dev(ggx, torch.float32), dev(ggv, torch.float32), dev(ggt, torch.float32))
+    torch.cuda.synchronize()
+    ref2 = conv.double_backward(prob, rowptr, col, vec32, x, th, gg, ggx, ggv, ggt)
+    for k in ("d_g", "d_x", "d_vec", "d_theta"):
+        assert rel(o2[k].cpu().numpy(), ref2[k]) < TOL_FP32, k
+
+
 def test_no_edges(T):
     import torch
     graph = (np.zeros(11, dtype=np.int32), np.zeros(0, dtype=np.int32), np.zeros((0, 3)))
