@@ -139,23 +139,4 @@ __global__ void __launch_bounds__(1024) k_build_work_list(int nc, const int* __r
   if (threadIdx.x == 0) *counter = 0;
 }
 
-// zero the state rows of the chunk's multi-piece nodes (their pieces add atomically);
-// recv: A blocks (rows 2l3+1 per node, Kb columns), else B blocks (2l1+1, Kx)
-__global__ void k_zero_heavy_rows(const __grid_constant__ DevPlan pl, int nc, const int* __restrict__ extra,
-                                  bool recv, float* __restrict__ out, float* __restrict__ out0) {
-  for (int i = blockIdx.x; i < nc; i += gridDim.x) {
-    if (extra[i + 1] == extra[i]) continue;
-    const int nb = recv ? pl.n_out : pl.n_in;
-    for (int b = 0; b < nb; ++b) {
-      const int rows = 2 * (recv ? pl.out_l[b] : pl.in_l[b]) + 1;
-      const int width = recv ? pl.Kb[b] : pl.Kx[b];
-      const size_t base = size_t(nc) * (recv ? pl.a_pref[b] : pl.b_pref[b]) + size_t(i) * rows * width;
-      for (int o = threadIdx.x; o < rows * width; o += blockDim.x) {
-        out[base + o] = 0.f;
-        if (out0) out0[base + o] = 0.f;
-      }
-    }
-  }
-}
-
 }  // namespace tpc

@@ -83,13 +83,13 @@ __device__ __forceinline__ void ffma2_bcast(float2& a, float2 b, float t) { a = 
 // one path, all channel tiles of the warp's node.  The radial state is kept as
 // float2 pairs of consecutive radial indices, so the outer products b (x) T run
 // as paired FMAs; shared-memory strides are the path's own compile-time widths.
-template <int L1, int L2, int L3, int RM, int CPL, bool RECV, bool DBL, bool P1>
+template <int L1, int L2, int L3, int RM, int CPL, bool RECV, bool DBL, bool P1, bool ADD>
 __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q, const WnLay& L, float* ws, int nl,
                                              int nc, int a0, int a1, const int* __restrict__ nbr,
                                              const int* __restrict__ perm, const float* __restrict__ vec,
                                              const float* __restrict__ ggv, const float* __restrict__ src,
                                              const float* __restrict__ src1, float* __restrict__ out,
-                                             float* __restrict__ out0, bool split) {
+                                             float* __restrict__ out0) {
   using TR = Tri<L1, L2, L3>;
   constexpr int N2 = TR::N2, NMZ = TR::NMZ, NMP = (NMZ + 3) & ~3;
   constexpr int NI = RECV ? TR::N1 : TR::N3;  // staged floats per channel
@@ -272,7 +272,7 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
           for (int i = 0; i < NO; ++i) {
             const float2 v = acc[((part * CPL + h) * NK2 + kp) * NO + i];
             float* d = dst + base + size_t(i) * Kq + ch;
-            if (split) {  // one piece of a long segment: add into the zeroed rows
+            if constexpr (ADD) {  // a further piece of a long segment: add onto the first piece's rows
               if (2 * kp < pl.R) atomicAdd(d + size_t(2 * kp) * c, v.x);
               if (2 * kp + 1 < pl.R) atomicAdd(d + size_t(2 * kp + 1) * c, v.y);
             } else {
@@ -292,9 +292,9 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
 // order, so the resident warps share one or two path bodies in the instruction
 // caches.  Second (EXTRA = true): a persistent grid whose warps claim the
 // further pieces of long segments, path-major, from *counter (list `extra`,
-// see graph.cuh); it ends at once when no segment is split.  A node with one
-// piece stores its state rows; a split node's pieces add into rows zeroed
-// beforehand.
+// see graph.cuh); it ends at once when no segment is split.  Every node's
+// first piece stores its state rows (first launch); the further pieces add onto
+// them (second launch, which starts after the first has finished).
 // RECV: ptr = rowptr, nbr = col (edge id = CSR position); else ptr = s_rowptr,
 // nbr = s_recv, perm = sender-sorted position -> edge id.
 template <int RM, int LF, int CPL, bool RECV, bool DBL, bool P1, bool EXTRA>
@@ -335,14 +335,13 @@ __global__ void __launch_bounds__(32 * kWnWarps, DBL && RECV ? 3 : 4)
     }
     const int s0 = ptr[n0 + nl], s1 = ptr[n0 + nl + 1];
     const int a0 = s0 + k * seg, a1 = min(s1, a0 + seg);
-    const bool split = s1 - s0 > seg;
     const DevPath& q = pl.path[p];
     switch (triple_id(q.l1, q.l2, q.l3)) {
 #define TPC_CASE(a, b, c)                                                                                        \
   case triple_id(a, b, c):                                                                                       \
     if constexpr (a <= LF && c <= LF)                                                                            \
-      wn_chan_path<a, b, c, RM, CPL, RECV, DBL, P1>(pl, q, L, ws, nl, nc, a0, a1, nbr, perm, vec, ggv, src, src1, \
-                                                    out, out0, split);                                           \
+      wn_chan_path<a, b, c, RM, CPL, RECV, DBL, P1, EXTRA>(pl, q, L, ws, nl, nc, a0, a1, nbr, perm, vec, ggv, src, \
+                                                           src1, out, out0);                                     \
     break;
       TPC_FOR_EACH_TRIPLE(TPC_CASE)
 #undef TPC_CASE

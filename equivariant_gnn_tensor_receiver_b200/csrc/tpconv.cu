@@ -374,13 +374,6 @@ int piece_edges(int64_t N, int64_t E) {
   const int64_t mean = N > 0 ? (E + N - 1) / N : 0;
   return int(std::max<int64_t>(256, 4 * mean));
 }
-// zero the state rows of the chunk's split nodes (their pieces add atomically)
-cudaError_t zero_split_rows(const DevPlan& d, int nc, const WorkList& wl, bool recv, float* out, float* out0,
-                            cudaStream_t s) {
-  k_zero_heavy_rows<<<unsigned(std::max(1, std::min(nc, 1184))), 128, 0, s>>>(d, nc, wl.extra, recv, out, out0);
-  return cudaGetLastError();
-}
-
 // ---- validate mode: the graph is checked on the device before any stream runs ----
 __device__ int g_graph_error;
 
@@ -539,12 +532,11 @@ int tpconv_forward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t*
       PhaseScope ps(TPCONV_PHASE_FWD_EDGE, s);
       const WorkList wl = work_list(L, workspace, 0, L.chunk_nodes);
       const int seg = piece_edges(N, E);
-      if (build_work_list(wl, L, rowptr, int(r0), nc, seg, s) || zero_split_rows(d, nc, wl, true, A, nullptr, s))
-        return TPCONV_ERR_CUDA;
+      if (build_work_list(wl, L, rowptr, int(r0), nc, seg, s)) return TPCONV_ERR_CUDA;
       if (TPC_WN_CALL_CPL(d, launch_wn_fwd, d, int(r0), nc, rowptr, col, edge_vec, x, A, wl.extra, wl.counter, seg,
                           s))
         return TPCONV_ERR_CUDA;
-      note(TPCONV_PHASE_FWD_EDGE, 4);  // list, zeroed split rows, two stream launches
+      note(TPCONV_PHASE_FWD_EDGE, 3);  // list, two stream launches
     }
     {
       PhaseScope ps(TPCONV_PHASE_FWD_NODE, s);
@@ -616,13 +608,11 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
         PhaseScope ps(TPCONV_PHASE_BWD_EDGE_S, s);
         const WorkList wl = work_list(L, workspace, 2, L.chunk_nodes);
         const int seg = piece_edges(N, E);
-        if (build_work_list(wl, L, s_rowptr, int(s0), nc, seg, s) ||
-            zero_split_rows(d, nc, wl, false, S_, nullptr, s))
-          return TPCONV_ERR_CUDA;
+        if (build_work_list(wl, L, s_rowptr, int(s0), nc, seg, s)) return TPCONV_ERR_CUDA;
         if (TPC_WN_CALL_CPL(d, launch_wn_send, d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, g, S_, wl.extra,
                             wl.counter, seg, s))
           return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_BWD_EDGE_S, 4);  // list, zeroed split rows, two stream launches
+        note(TPCONV_PHASE_BWD_EDGE_S, 3);  // list, two stream launches
       }
       {
         PhaseScope ps(TPCONV_PHASE_BWD_NODE_X, s);
@@ -687,13 +677,11 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
         PhaseScope ps(TPCONV_PHASE_DBL_EDGE_A, s);
         const WorkList wl = work_list(L, workspace, 0, L.chunk_nodes);
         const int seg = piece_edges(N, E);
-        if (build_work_list(wl, L, rowptr, int(r0), nc, seg, s) ||
-            zero_split_rows(d, nc, wl, true, A1, has_t ? A0 : nullptr, s))
-          return TPCONV_ERR_CUDA;
+        if (build_work_list(wl, L, rowptr, int(r0), nc, seg, s)) return TPCONV_ERR_CUDA;
         if (TPC_WN_CALL(d, launch_wn_dbla, d, int(r0), nc, rowptr, col, edge_vec, gg_vec, x, gg_x, A1,
                         has_t ? A0 : nullptr, wl.extra, wl.counter, seg, s))
           return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_DBL_EDGE_A, 4);  // list, zeroed split rows, two stream launches
+        note(TPCONV_PHASE_DBL_EDGE_A, 3);  // list, two stream launches
       }
       PhaseScope ps(TPCONV_PHASE_DBL_NODE_A, s);
       if (node_mix_forward(plan, int(r0), nc, A1, theta, t_hi, t_lo, d_g, s, 0)) return TPCONV_ERR_CUDA;
@@ -743,12 +731,11 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
         float* B0u = (has_x1 || has_t) ? B0 : nullptr;
         const WorkList wl = work_list(L, workspace, 2, L.chunk_nodes);
         const int seg = piece_edges(N, E);
-        if (build_work_list(wl, L, s_rowptr, int(s0), nc, seg, s) || zero_split_rows(d, nc, wl, false, B1, B0u, s))
-          return TPCONV_ERR_CUDA;
+        if (build_work_list(wl, L, s_rowptr, int(s0), nc, seg, s)) return TPCONV_ERR_CUDA;
         if (TPC_WN_CALL(d, launch_wn_dbls, d, int(s0), nc, s_rowptr, perm, s_recv, edge_vec, gg_vec, g, B1, B0u,
                         wl.extra, wl.counter, seg, s))
           return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_DBL_EDGE_S, 4);  // list, zeroed split rows, two stream launches
+        note(TPCONV_PHASE_DBL_EDGE_S, 3);  // list, two stream launches
       }
       PhaseScope ps(TPCONV_PHASE_DBL_NODE_X, s);
       float* dx1 = has_v ? d_x : nullptr;
