@@ -17,7 +17,9 @@ What it computes (all fp64, numpy):
               abstract of "Sobek" (arXiv 2607.18074): per-edge weights
               W_e = sum_k b_ek Theta_k are materialised, per-edge messages are
               formed and scatter-added to receivers; backward and double
-              backward are the explicit adjoints of that schedule.
+              backward are the explicit adjoints of that schedule.  Two
+              operator families: "full" (Theta[p] is R x C_in x C_out) and
+              "channelwise" (Theta[p] is R x C, W_e[p] diagonal).
 
 Sources: "Sobek: streaming edge-conditioned equivariant tensor-product
 convolution" (arXiv 2607.18074), abstract -- the operator (radial projection,

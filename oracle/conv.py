@@ -11,6 +11,14 @@ mixing; the exact formula is a reading):
     W_e[p]            = sum_k b_k(|v_e|) Theta[p][k]              (C_in x C_out)
     T_e[p, u, m3]     = sum_{m1, m2} C_p[m1, m2, m3] x[send(e), i1, u, m1] Y_{l2, m2}(v_e)
 
+Second operator family ("channelwise"; the abstract counts two operator
+families without naming them, the reading taken is the channel-wise product):
+every path keeps each channel on its own, W_e[p] = diag(sum_k b_k Theta[p][k])
+with Theta[p] of shape R x C (C_in = C_out = C), so
+
+    out[r, i3, u, m3] = sum_e sum_{p -> i3} w_e[p, u] * T_e[p, u, m3],
+    w_e[p, u]         = sum_k b_k(|v_e|) Theta[p][k, u].
+
 The abstract names the conventional schedule as the one that materialises
 edge-specific weights, messages and adjoints; this module is exactly that
 schedule (edge chunks keep host memory bounded): W_e and the message of every
@@ -43,6 +51,7 @@ class Problem:
     R: int
     radial: str = "bessel"            # "gaussian" | "bessel"
     radial_params: tuple = (5.0,)     # (r_min, r_max) | (r_cut,)
+    family: str = "full"              # "full" | "channelwise"
     paths: list = field(init=False)
     dim_in: int = field(init=False)
     dim_out: int = field(init=False)
@@ -50,15 +59,47 @@ class Problem:
     theta_numel: int = field(init=False)
 
     def __post_init__(self):
-        self.paths = _irreps.paths(self.irreps_in, self.l_sh_max, self.irreps_out, self.R)
+        self.paths = _irreps.paths(self.irreps_in, self.l_sh_max, self.irreps_out, self.R, self.family)
         self.dim_in = _irreps.dim(_irreps.parse(self.irreps_in))
         self.dim_out = _irreps.dim(_irreps.parse(self.irreps_out))
         self.n_sh = (self.l_sh_max + 1) ** 2
-        self.theta_numel = _irreps.theta_numel(self.paths, self.R)
+        self.theta_numel = _irreps.theta_numel(self.paths, self.R, self.family)
+
+    @property
+    def channelwise(self) -> bool:
+        return self.family == "channelwise"
+
+    def theta_size(self, p) -> int:
+        return self.R * p.c_in * (1 if self.channelwise else p.c_out)
 
     def theta_block(self, theta, p):
-        n = self.R * p.c_in * p.c_out
-        return theta[p.theta_off:p.theta_off + n].reshape(self.R, p.c_in, p.c_out)
+        """Theta[p]: (R, C_in, C_out), or (R, C) for the channel-wise family."""
+        blk = theta[p.theta_off:p.theta_off + self.theta_size(p)]
+        return blk.reshape(self.R, p.c_in) if self.channelwise else blk.reshape(self.R, p.c_in, p.c_out)
+
+
+# Edge weights and their uses, per family.  Full: W (E, C_in, C_out); channel-wise:
+# the diagonal w (E, C) of the same matrix.
+
+def _weights(prob, b, Th):
+    return np.einsum('ek,ku->eu', b, Th) if prob.channelwise else np.einsum('ek,kuw->euw', b, Th)
+
+
+def _message(prob, W, T):
+    """msg[e, w, m3] = sum_u W[e, u, w] T[e, u, m3]."""
+    return W[:, :, None] * T if prob.channelwise else np.einsum('euw,euk->ewk', W, T, optimize=True)
+
+
+def _weight_adjoint(prob, T, gr):
+    """dW = d<g, msg>/dW  (full: (E, C_in, C_out); channel-wise: its diagonal (E, C))."""
+    if prob.channelwise:
+        return np.einsum('euk,euk->eu', T, gr)
+    return np.einsum('euk,ewk->euw', T, gr, optimize=True)
+
+
+def _message_adjoint(prob, W, gr):
+    """dT[e, u, m3] = sum_w W[e, u, w] g_r[w, m3]."""
+    return W[:, :, None] * gr if prob.channelwise else np.einsum('euw,ewk->euk', W, gr, optimize=True)
 
 
 def receivers_of(rowptr) -> np.ndarray:
@@ -108,10 +149,10 @@ def forward_core(prob: Problem, N: int, send, recv, x, Y, b, theta):
         s, r = send[e0:e1], recv[e0:e1]
         for p in prob.paths:
             C = _so3.real_cg(p.l1, p.l2, p.l3)
-            W = np.einsum('ek,kuw->euw', b[e0:e1], prob.theta_block(theta, p))   # edge weights
+            W = _weights(prob, b[e0:e1], prob.theta_block(theta, p))              # edge weights
             xs = _in_block(prob, x, s, p)
             T = np.einsum('ijk,eui,ej->euk', C, xs, _sh_block(Y[e0:e1], p.l2), optimize=True)
-            msg = np.einsum('euw,euk->ewk', W, T, optimize=True)                   # edge message
+            msg = _message(prob, W, T)                                             # edge message
             n3 = 2 * p.l3 + 1
             np.add.at(out[:, p.out_off:p.out_off + p.c_out * n3], r, msg.reshape(len(r), -1))
     return out
@@ -129,17 +170,20 @@ def backward_core(prob: Problem, N: int, send, recv, x, Y, b, theta, g):
         for p in prob.paths:
             C = _so3.real_cg(p.l1, p.l2, p.l3)
             Th = prob.theta_block(theta, p)
-            W = np.einsum('ek,kuw->euw', b[e0:e1], Th)
+            W = _weights(prob, b[e0:e1], Th)
             xs = _in_block(prob, x, s, p)
             Ys = _sh_block(Y[e0:e1], p.l2)
             T = np.einsum('ijk,eui,ej->euk', C, xs, Ys, optimize=True)
             gr = _out_block(prob, g, r, p)
-            dW = np.einsum('euk,ewk->euw', T, gr, optimize=True)                  # weight adjoint
-            n = prob.R * p.c_in * p.c_out
-            dtheta[p.theta_off:p.theta_off + n] += np.einsum('ek,euw->kuw', b[e0:e1], dW,
-                                                             optimize=True).reshape(-1)
-            db[e0:e1] += np.einsum('kuw,euw->ek', Th, dW, optimize=True)
-            dT = np.einsum('euw,ewk->euk', W, gr, optimize=True)                  # message adjoint
+            dW = _weight_adjoint(prob, T, gr)                                     # weight adjoint
+            n = prob.theta_size(p)
+            # dTheta[k] = sum_e b_ek dW_e and db_ek = <Theta[k], dW_e>
+            dtheta[p.theta_off:p.theta_off + n] += np.einsum('ek,e...->k...', b[e0:e1], dW).reshape(-1)
+            if prob.channelwise:
+                db[e0:e1] += np.einsum('ku,eu->ek', Th, dW)
+            else:
+                db[e0:e1] += np.einsum('kuw,euw->ek', Th, dW, optimize=True)
+            dT = _message_adjoint(prob, W, gr)                                    # message adjoint
             dxs = np.einsum('ijk,ej,euk->eui', C, Ys, dT, optimize=True)
             n1 = 2 * p.l1 + 1
             np.add.at(dx[:, p.in_off:p.in_off + p.c_in * n1], s, dxs.reshape(len(s), -1))

@@ -67,7 +67,14 @@ class Path:
     theta_off: int
 
 
-def paths(irreps_in: str, l_sh_max: int, irreps_out: str, R: int) -> list[Path]:
+def paths(irreps_in: str, l_sh_max: int, irreps_out: str, R: int, family: str = "full") -> list[Path]:
+    """Paths in canonical order (output block, input block, l2) with their Theta offsets.
+
+    family "full": Theta[p] is R x C_in x C_out (every input channel mixes into every output
+    channel); "channelwise": Theta[p] is R x C, one weight per radial function and channel,
+    which needs C_in = C_out on every path."""
+    if family not in ("full", "channelwise"):
+        raise ValueError(f"unknown operator family {family!r}")
     bin_, bout = parse(irreps_in), parse(irreps_out)
     oin, oout = offsets(bin_), offsets(bout)
     out, toff = [], 0
@@ -78,10 +85,12 @@ def paths(irreps_in: str, l_sh_max: int, irreps_out: str, R: int) -> list[Path]:
                     continue
                 if b1.p * (-1) ** l2 != b3.p:
                     continue
+                if family == "channelwise" and b1.mul != b3.mul:
+                    raise ValueError("the channel-wise product needs equal input and output multiplicities")
                 out.append(Path(i1, l2, i3, b1.l, b3.l, b1.mul, b3.mul, oin[i1], oout[i3], toff))
-                toff += R * b1.mul * b3.mul
+                toff += R * b1.mul * (b3.mul if family == "full" else 1)
     return out
 
 
-def theta_numel(ps: list[Path], R: int) -> int:
-    return sum(R * p.c_in * p.c_out for p in ps)
+def theta_numel(ps: list[Path], R: int, family: str = "full") -> int:
+    return sum(R * p.c_in * (p.c_out if family == "full" else 1) for p in ps)
