@@ -48,7 +48,8 @@ WORKLOADS = {
 
 
 def workload(args):
-    return WORKLOADS[args.config].format(d=args.degree or 25)
+    w = WORKLOADS[args.config].format(d=args.degree or 25)
+    return w + ", channel-wise weights" if args.family == "channelwise" else w
 METRIC = "edges/s (fwd + bwd + double bwd step)"
 L2_BYTES = 126 * 1024 * 1024
 FP32_LANES_PER_SM = 128
@@ -63,6 +64,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="mace")
     ap.add_argument("--gemm", default="fp32", choices=["fp32", "tf32", "simt"])
+    ap.add_argument("--family", default="full", choices=["full", "channelwise"],
+                    help="operator family: fully connected or channel-wise per-path weights")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--degree", type=float, default=None, help="mean degree of the sweep workload")
     ap.add_argument("--workspace-cap", type=int, default=None,
@@ -180,12 +183,20 @@ def cpu_cores():
     return int(n)
 
 
-def oracle_sample(cfg, graph, n_recv, seed=100):
+def theta_segments(paths, R, family):
+    """Normal Theta blocks per path: R x C_in x C_out (std 1/sqrt(R C_in)) or R x C (std 1/sqrt(R))."""
+    get = (lambda p, k: p[k]) if isinstance(paths[0], dict) else (lambda p, k: getattr(p, k))
+    if family == "channelwise":
+        return [(R * get(p, "c_in"), 1 / np.sqrt(R)) for p in paths]
+    return [(R * get(p, "c_in") * get(p, "c_out"), 1 / np.sqrt(R * get(p, "c_in"))) for p in paths]
+
+
+def oracle_sample(cfg, graph, n_recv, seed=100, family="full"):
     """Oracle step (fwd + bwd + double bwd) on the edges of the first n_recv receivers."""
     from oracle import conv
     c = W.CONFIGS[cfg]
     prob = conv.Problem(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], c["radial"],
-                        tuple(c["radial_params"]))
+                        tuple(c["radial_params"]), family=family)
     rowptr, col, vec = graph
     e1 = int(rowptr[n_recv])
     rp = np.asarray(rowptr[:n_recv + 1], dtype=np.int64)
@@ -195,7 +206,7 @@ def oracle_sample(cfg, graph, n_recv, seed=100):
     vec = vec[:e1]
     N = len(nodes)
     x = W.normal((N, prob.dim_in), seed)
-    th = W.theta([(prob.R * p.c_in * p.c_out, 1 / np.sqrt(prob.R * p.c_in)) for p in prob.paths], seed + 1)
+    th = W.theta(theta_segments(prob.paths, prob.R, family), seed + 1)
     g = np.zeros((n_recv, prob.dim_out))
     g[:] = W.normal((n_recv, prob.dim_out), seed + 2)
     ggx = W.normal((N, prob.dim_in), seed + 3)
@@ -238,7 +249,7 @@ def run_reference(args):
         return
     graph = W.graph_for(args.config, 0)
     n_recv = 8
-    step, e = oracle_sample(args.config, graph, n_recv)
+    step, e = oracle_sample(args.config, graph, n_recv, family=args.family)
     for _ in range(args.warmup):
         step()
     t0 = time.perf_counter()
@@ -277,14 +288,13 @@ def run_ours(args):
     N, E = len(rowptr) - 1, len(col)
     cap = args.workspace_cap if args.workspace_cap is not None else (8 << 30 if args.config == "capacity" else 0)
     plan = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], radial=c["radial"],
-                  radial_params=c["radial_params"], gemm=args.gemm, workspace_cap=cap)
+                  radial_params=c["radial_params"], gemm=args.gemm, workspace_cap=cap, family=args.family)
     f32 = torch.float32
     pin = lambda a, dt=f32: torch.as_tensor(np.ascontiguousarray(a), dtype=dt).pin_memory()
     host = {
         "rowptr": pin(rowptr, torch.int32), "col": pin(col, torch.int32), "vec": pin(vec),
         "x": pin(W.normal((N, plan.dim_in), 10 + rank)),
-        "theta": pin(W.theta([(plan.R * p["c_in"] * p["c_out"], 1 / np.sqrt(plan.R * p["c_in"]))
-                              for p in plan.paths], 11 + rank)),
+        "theta": pin(W.theta(theta_segments(plan.paths, plan.R, args.family), 11 + rank)),
         "g": pin(W.normal((N, plan.dim_out), 12 + rank)),
         "gg_x": pin(W.normal((N, plan.dim_in), 13 + rank)),
         "gg_vec": pin(W.normal((E, 3), 14 + rank)),
@@ -397,7 +407,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        stepc, ec = oracle_sample(args.config, (rowptr, col, vec), 4)
+        stepc, ec = oracle_sample(args.config, (rowptr, col, vec), 4, family=args.family)
         stepc()
         t0 = time.perf_counter()
         reps = 0
@@ -415,6 +425,7 @@ def run_ours(args):
             "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": step_ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": workload(args), "workspace_cap": cap, "nodes_per_gpu": N, "edges_per_gpu": E, "gemm": args.gemm,
+                       "family": args.family,
                        "step": "graph transpose + fwd + bwd(dx,dTheta,dvec) + double bwd(gg_x,gg_vec)",
                        "l2": "256 MiB buffer zeroed before every timed step, outside the events",
                        "parallelism": f"{world} independent replicas (one graph per rank)"},

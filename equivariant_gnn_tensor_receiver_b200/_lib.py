@@ -22,6 +22,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "bad irreps", 3: "unsupported", 4: 
           5: "CUDA error", 6: "graph invalid", 7: "timeout", 8: "internal"}
 RADIAL = {"gaussian": 0, "bessel": 1}
 GEMM = {"fp32": 0, "tf32": 1, "bf16": 2, "simt": 3}
+FAMILY = {"full": 0, "channelwise": 1}
 OP_FORWARD, OP_BACKWARD, OP_DOUBLE_BACKWARD, OP_TRANSPOSE = 0, 1, 2, 3
 
 
@@ -33,7 +34,8 @@ class TPConvError(RuntimeError):
 
 class Options(ctypes.Structure):
     _fields_ = [("radial", ctypes.c_int), ("radial_p0", ctypes.c_double), ("radial_p1", ctypes.c_double),
-                ("gemm", ctypes.c_int), ("workspace_cap", ctypes.c_size_t), ("validate", ctypes.c_int)]
+                ("gemm", ctypes.c_int), ("workspace_cap", ctypes.c_size_t), ("validate", ctypes.c_int),
+                ("family", ctypes.c_int)]
 
 
 _lib = None
@@ -102,7 +104,7 @@ class Plan:
     """Owner of a ``tpconv_plan*``."""
 
     def __init__(self, irreps_in, l_sh_max, irreps_out, R, radial="bessel", radial_params=(5.0,), gemm="fp32",
-                 workspace_cap=0, validate=False):
+                 workspace_cap=0, validate=False, family="full"):
         o = default_options()
         o.radial = RADIAL[radial]
         o.radial_p0 = float(radial_params[0])
@@ -110,12 +112,14 @@ class Plan:
         o.gemm = GEMM[gemm]
         o.workspace_cap = int(workspace_cap)
         o.validate = int(bool(validate))
+        o.family = FAMILY[family]
         h = _P()
         _check("tpconv_plan_create",
                lib().tpconv_plan_create(ctypes.byref(h), irreps_in.encode(), int(l_sh_max), irreps_out.encode(),
                                         int(R), ctypes.byref(o)))
         self.handle = h
         self.irreps_in, self.irreps_out, self.l_sh_max, self.R = irreps_in, irreps_out, l_sh_max, R
+        self.family = family
         self.options = o
         a = [ctypes.c_int() for _ in range(4)]
         t = ctypes.c_size_t()

@@ -127,8 +127,9 @@ class _ConvBwdFn(torch.autograd.Function):
 class TPConv(torch.nn.Module):
     """The streaming CG tensor-product convolution as a torch module.
 
-    Holds Theta ([P][R][C_in][C_out], one normal block per path with standard
-    deviation 1/sqrt(R C_in)) as a parameter; ``forward(x, graph)`` returns
+    Holds Theta ([P][R][C_in][C_out], or [P][R][C] with ``family="channelwise"``;
+    one normal block per path with standard deviation 1/sqrt(R C_in), 1/sqrt(R)
+    channel-wise) as a parameter; ``forward(x, graph)`` returns
     out[N][dim_out] for the receiver-sorted ``Graph`` (its ``edge_vec`` may
     require grad).  Differentiable twice in x, Theta and the edge vectors.
     """
@@ -136,8 +137,9 @@ class TPConv(torch.nn.Module):
     def __init__(self, irreps_in, l_sh_max, irreps_out, R, device="cuda", **plan_options):
         super().__init__()
         self.plan = L.Plan(irreps_in, l_sh_max, irreps_out, R, **plan_options)
-        blocks = [torch.randn(self.plan.R * p["c_in"] * p["c_out"]) / (self.plan.R * p["c_in"]) ** 0.5
-                  for p in self.plan.paths]
+        cw = self.plan.family == "channelwise"
+        blocks = [torch.randn(self.plan.R * p["c_in"] * (1 if cw else p["c_out"]))
+                  / (self.plan.R * (1 if cw else p["c_in"])) ** 0.5 for p in self.plan.paths]
         self.theta = torch.nn.Parameter(torch.cat(blocks).to(device=device, dtype=torch.float32))
 
     def forward(self, x, graph: Graph):

@@ -225,6 +225,7 @@ void tpconv_default_options(tpconv_options* opt) {
   opt->gemm = TPCONV_GEMM_FP32;
   opt->workspace_cap = 0;
   opt->validate = 0;
+  opt->family = TPCONV_FAMILY_FULL;
 }
 
 const char* tpconv_status_string(int st) {
@@ -256,6 +257,7 @@ int tpconv_plan_create(tpconv_plan** out, const char* irreps_in, int l_sh_max,
     return TPCONV_ERR_INVALID_ARG;
   if (o.gemm < TPCONV_GEMM_FP32 || o.gemm > TPCONV_GEMM_SIMT) return TPCONV_ERR_INVALID_ARG;
   if (o.gemm == TPCONV_GEMM_BF16) return TPCONV_ERR_UNSUPPORTED;  // reserved, not built
+  if (o.family != TPCONV_FAMILY_FULL && o.family != TPCONV_FAMILY_CHANNELWISE) return TPCONV_ERR_INVALID_ARG;
   if (o.radial == TPCONV_RADIAL_BESSEL_COS && !(o.radial_p0 > 0)) return TPCONV_ERR_INVALID_ARG;
   if (o.radial == TPCONV_RADIAL_GAUSSIAN && !(o.radial_p1 > o.radial_p0)) return TPCONV_ERR_INVALID_ARG;
 
@@ -317,6 +319,10 @@ int tpconv_plan_create(tpconv_plan** out, const char* irreps_in, int l_sh_max,
           delete p;
           return TPCONV_ERR_UNSUPPORTED;
         }
+        if (o.family == TPCONV_FAMILY_CHANNELWISE && b1.mul != b3.mul) {  // one weight per channel
+          delete p;
+          return TPCONV_ERR_INVALID_ARG;
+        }
         DevPath& q = d.path[P++];
         q.l1 = int8_t(b1.l);
         q.l2 = int8_t(l2);
@@ -332,9 +338,10 @@ int tpconv_plan_create(tpconv_plan** out, const char* irreps_in, int l_sh_max,
         d.Kb[i3] += R * b1.mul;
         q.kxoff = d.Kx[i1];
         d.Kx[i1] += R * b3.mul;
-        toff += int64_t(R) * b1.mul * b3.mul;
+        toff += int64_t(R) * b1.mul * (o.family == TPCONV_FAMILY_CHANNELWISE ? 1 : b3.mul);
       }
   d.P = P;
+  d.family = o.family;
   d.rm = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
   int sm = 0, sm2 = 0;
   for (int i = 0; i < P; ++i) {

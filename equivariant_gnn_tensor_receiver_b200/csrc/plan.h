@@ -119,6 +119,7 @@ struct DevPlan {
   int wn_smem_f, wn_smem_s;         // dynamic smem bytes: receiver / sender form, first order
   int wn_smem_f2, wn_smem_s2;       // the same, second order
   int wn_smem_adj, wn_smem_dadj;    // receiver adjoint streams, first / second order
+  int family;                       // TPCONV_FAMILY_*: Theta[p] is R x C_in x C_out or R x C
   DevPath path[kMaxPaths];
 };
 

@@ -19,6 +19,7 @@
 #include <vector>
 
 #include "gemm_simt.cuh"
+#include "channelwise.h"
 #include "dtheta.h"
 #include "gemm_tc.h"
 #include "graph.cuh"
@@ -133,8 +134,10 @@ cudaError_t prep_theta_T(const tpconv_plan* plan, const float* theta, float* hi,
 }
 
 bool use_tc(const tpconv_plan* plan) {
-  return plan->opt.gemm == TPCONV_GEMM_FP32 || plan->opt.gemm == TPCONV_GEMM_TF32;
+  return plan->dp.family == TPCONV_FAMILY_FULL &&
+         (plan->opt.gemm == TPCONV_GEMM_FP32 || plan->opt.gemm == TPCONV_GEMM_TF32);
 }
+bool channelwise(const tpconv_plan* plan) { return plan->dp.family == TPCONV_FAMILY_CHANNELWISE; }
 
 // out[r0 : r0+nc] = A . Theta (mode 0) or += (mode 1), per output block.  With
 // thT (Theta^T hi, lo) the tensor-core GEMM runs, else the FFMA GEMM.
@@ -207,6 +210,7 @@ class ForkJoin {
 cudaError_t node_mix_forward(const tpconv_plan* plan, int r0, int nc, const float* A, const float* theta,
                              const float* thT_hi, const float* thT_lo, float* out, cudaStream_t st, int mode = 0) {
   const DevPlan& d = plan->dp;
+  if (channelwise(plan)) return cw_forward(d, r0, nc, A, theta, out, mode, st);
   ForkJoin fj(st);
   for (int i3 = 0; i3 < d.n_out; ++i3) {
     cudaStream_t si = fj.stream(i3);
@@ -285,6 +289,7 @@ cudaError_t prep_tc_theta(const tpconv_plan* plan, const float* theta, float* re
 cudaError_t node_mix_adjoint(const tpconv_plan* plan, int r0, int nc, const float* g, const float* theta,
                              const TcTheta* tc, float* gpack, float* G, cudaStream_t st) {
   const DevPlan& d = plan->dp;
+  if (channelwise(plan)) return cw_adjoint(d, r0, nc, g, theta, G, st);
   ForkJoin fj(st);
   for (int i3 = 0; i3 < d.n_out; ++i3) {
     if (d.Kb[i3] == 0) continue;
@@ -319,6 +324,10 @@ cudaError_t node_mix_sender(const tpconv_plan* plan, int s0, int nc, const float
                             const float* theta, const TcTheta* tc, float* dx, float* dtheta, cudaStream_t st) {
   const DevPlan& d = plan->dp;
   cudaError_t e;
+  if (channelwise(plan)) {
+    if (dx && (e = cw_dx(d, s0, nc, B, theta, dx, st))) return e;
+    return dtheta ? cw_dtheta(d, s0, nc, x, B, nullptr, nullptr, dtheta, st) : cudaSuccess;
+  }
   ForkJoin fj(st);
   if (dx) {
     for (int i1 = 0; i1 < d.n_in; ++i1) {
@@ -584,7 +593,7 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
       {
         PhaseScope ps(TPCONV_PHASE_BWD_NODE_G, s);
         if (node_mix_adjoint(plan, int(r0), nc, g, theta, tcp, gpack, S_, s)) return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_BWD_NODE_G, 2 * d.n_out);
+        note(TPCONV_PHASE_BWD_NODE_G, channelwise(plan) ? cw_launches_out(d) : 2 * d.n_out);
       }
       {
         PhaseScope ps(TPCONV_PHASE_BWD_EDGE_R, s);
@@ -617,7 +626,8 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
       {
         PhaseScope ps(TPCONV_PHASE_BWD_NODE_X, s);
         if (node_mix_sender(plan, int(s0), nc, S_, x, theta, tcp, dx, dtheta, s)) return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_BWD_NODE_X, int64_t(dx ? d.n_in : 0) + int64_t(dtheta ? 1 : 0));
+        const int64_t nx = channelwise(plan) ? cw_launches_in(d) : d.n_in;
+        note(TPCONV_PHASE_BWD_NODE_X, int64_t(dx ? nx : 0) + int64_t(dtheta ? (channelwise(plan) ? nx : 1) : 0));
       }
     }
   }
@@ -701,10 +711,11 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
       {
         PhaseScope ps(TPCONV_PHASE_OTHER, s);
         if (node_mix_adjoint(plan, int(r0), nc, g, theta, tc0p, gpack, G, s)) return TPCONV_ERR_CUDA;
-        note(TPCONV_PHASE_OTHER, 2 * d.n_out);
+        const int64_t na = channelwise(plan) ? cw_launches_out(d) : 2 * d.n_out;
+        note(TPCONV_PHASE_OTHER, na);
         if (has_t) {
           if (node_mix_adjoint(plan, int(r0), nc, g, gg_theta, tc1p, gpack, Gt, s)) return TPCONV_ERR_CUDA;
-          note(TPCONV_PHASE_OTHER, 2 * d.n_out);
+          note(TPCONV_PHASE_OTHER, na);
         }
       }
       PhaseScope ps(TPCONV_PHASE_DBL_EDGE_R, s);
@@ -745,10 +756,13 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
       float* dt0 = has_x1 ? d_theta : nullptr;
       if (dx0 && node_mix_sender(plan, int(s0), nc, B0, gg_x, gg_theta, tc1p, dx0, nullptr, s)) return TPCONV_ERR_CUDA;
       // d_theta = x^T B1 + gg_x^T B0 in one pass
-      if ((dt1 || dt0) && dtheta_accumulate(d, int(s0), nc, dt1 ? x : nullptr, dt1 ? B1 : nullptr, dt0 ? gg_x : nullptr,
-                                            dt0 ? B0 : nullptr, d_theta, s))
+      if ((dt1 || dt0) &&
+          (channelwise(plan) ? cw_dtheta : dtheta_accumulate)(d, int(s0), nc, dt1 ? x : nullptr, dt1 ? B1 : nullptr,
+                                                              dt0 ? gg_x : nullptr, dt0 ? B0 : nullptr, d_theta, s))
         return TPCONV_ERR_CUDA;
-      note(TPCONV_PHASE_DBL_NODE_X, int64_t(dx1 ? d.n_in : 0) + int64_t(dx0 ? d.n_in : 0) + ((dt1 || dt0) ? 1 : 0));
+      const int64_t nx = channelwise(plan) ? cw_launches_in(d) : d.n_in;
+      note(TPCONV_PHASE_DBL_NODE_X,
+           int64_t(dx1 ? nx : 0) + int64_t(dx0 ? nx : 0) + ((dt1 || dt0) ? (channelwise(plan) ? nx : 1) : 0));
     }
   }
   return finish(cudaSuccess);

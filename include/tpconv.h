@@ -78,6 +78,21 @@ extern "C" {
 #define TPCONV_GEMM_BF16 2 /* reserved: plan creation returns UNSUPPORTED */
 #define TPCONV_GEMM_SIMT 3 /* plain fp32 FFMA (reference-precision mode)  */
 
+/* operator families (tpconv_options.family).  Both follow "Sobek: streaming
+ * edge-conditioned equivariant tensor-product convolution" (arXiv 2607.18074),
+ * abstract, which evaluates two operator families without naming them:
+ *   FULL         W_e[p] = sum_k b_k(|v_e|) Theta[p][k], a C_in x C_out matrix
+ *                (fully connected multiplicity mixing); Theta is
+ *                [P][R][C_in][C_out].
+ *   CHANNELWISE  W_e[p] = diag(sum_k b_k(|v_e|) Theta[p][k, :]): each channel
+ *                keeps its own weight; Theta is [P][R][C].  Every path needs
+ *                C_in = C_out, else plan creation returns
+ *                TPCONV_ERR_INVALID_ARG.  The edge streams are those of FULL;
+ *                the node-level contractions become per-channel sums.
+ * The path order and the CG coupling are the same for both. */
+#define TPCONV_FAMILY_FULL 0
+#define TPCONV_FAMILY_CHANNELWISE 1
+
 /* operations, for tpconv_workspace_size */
 #define TPCONV_OP_FORWARD 0
 #define TPCONV_OP_BACKWARD 1
@@ -93,9 +108,11 @@ typedef struct tpconv_options {
   int gemm;              /* TPCONV_GEMM_*                                     */
   size_t workspace_cap;  /* bytes of node-side state per chunk; 0 = no cap    */
   int validate;          /* 1: check the graph on the device first (syncs)    */
+  int family;            /* TPCONV_FAMILY_*                                   */
 } tpconv_options;
 
-/* Fill *opt with defaults: Bessel (r_cut 5), GEMM_FP32, no cap, no validation. */
+/* Fill *opt with defaults: Bessel (r_cut 5), GEMM_FP32, no cap, no validation,
+ * the FULL family. */
 void tpconv_default_options(tpconv_options* opt);
 
 /* Human-readable name of a status code (static storage; never NULL). */

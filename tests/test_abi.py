@@ -47,6 +47,31 @@ def test_plan_matches_oracle_path_table(T, name):
             p.l1, p.l2, p.l3, p.c_in, p.c_out, p.theta_off)
 
 
+@pytest.mark.parametrize("name", ["tiny", "mace", "wide"])
+def test_channelwise_plan_matches_oracle_path_table(T, name):
+    c = W.CONFIGS[name]
+    plan = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], radial=c["radial"],
+                  radial_params=c["radial_params"], family="channelwise")
+    prob = conv.Problem(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], c["radial"], c["radial_params"],
+                        family="channelwise")
+    assert (plan.n_paths, plan.theta_numel) == (len(prob.paths), prob.theta_numel)
+    assert [a["theta_offset"] for a in plan.paths] == [p.theta_off for p in prob.paths]
+    # the node-side state does not depend on the family
+    full = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], radial=c["radial"],
+                  radial_params=c["radial_params"])
+    L = T._lib
+    for op in (L.OP_FORWARD, L.OP_BACKWARD, L.OP_DOUBLE_BACKWARD):
+        a = L.tpconv_workspace_size(plan, op, 1000, 20000)
+        b = L.tpconv_workspace_size(full, op, 1000, 20000)
+        assert a <= b
+
+
+def test_channelwise_needs_equal_multiplicities(T):
+    with pytest.raises(T._lib.TPConvError) as e:
+        T.Plan("4x0e+2x1o", 1, "3x0e+2x1o", 2, family="channelwise")
+    assert e.value.status == 1
+
+
 def test_cg_table_matches_null_space_construction(T):
     worst = 0.0
     for l1 in range(4):
