@@ -143,9 +143,11 @@ __device__ __forceinline__ void tile(const DevPlan& pl, const DevPath& q, int u0
   }
 }
 
-// grid.x: tiles (p, u tile, n tile) over the plan's largest extents, grid.y: K splits
+// grid.x: tiles (p, u tile, n tile) over the plan's largest extents, grid.y: K splits.
+// A split holds about rows_per_split K rows: nodes x (2 l1 + 1) of its path, so the
+// CTAs of every path carry the same work and one wave ends together.
 __global__ void __launch_bounds__(kThreads, 2)
-    k_dtheta(const __grid_constant__ DevPlan pl, int s0, int nc, int ut, int nt, int nodes_per_split,
+    k_dtheta(const __grid_constant__ DevPlan pl, int s0, int nc, int ut, int nt, int rows_per_split,
              const float* __restrict__ xa, const float* __restrict__ Ba, const float* __restrict__ xb,
              const float* __restrict__ Bb, float* __restrict__ dtheta) {
   extern __shared__ __align__(16) float sm[];
@@ -154,8 +156,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   const DevPath& q = pl.path[p];
   const int u0 = (r / nt) * kTU, n0 = (r % nt) * kTN;
   if (u0 >= q.c_in || n0 >= pl.R * q.c_out) return;
+  const int n1 = 2 * q.l1 + 1;
+  const int nodes_per_split = max(1, (rows_per_split + n1 - 1) / n1);
+  if (int64_t(blockIdx.y) * nodes_per_split >= nc) return;
   const int sb = blockIdx.y * nodes_per_split, se = min(nc, sb + nodes_per_split);
-  if (sb >= se) return;
   switch (q.l1) {
     case 0: tile<1>(pl, q, u0, n0, sb, se, s0, nc, xa, Ba, xb, Bb, dtheta, sm); break;
     case 1: tile<3>(pl, q, u0, n0, sb, se, s0, nc, xa, Ba, xb, Bb, dtheta, sm); break;
@@ -176,12 +180,37 @@ cudaError_t dtheta_accumulate(const DevPlan& d, int s0, int nc, const float* xa,
   const int ut = (d.max_c_in + kTU - 1) / kTU;
   const int nt = (d.R * d.max_c_out + kTN - 1) / kTN;
   const int tiles = d.P * ut * nt;
-  // one wave of two CTAs per SM, each with at least 16 nodes of K
+  // One wave of two CTAs per SM with equal K rows per CTA: the rows of all
+  // (non-empty) tiles over the slots, grown until the split count fits.
   const int slots = 2 * 148;
-  const int splits = std::max(1, std::min(slots / tiles, (nc + 15) / 16));
-  const int per = (nc + splits - 1) / splits;
-  dim3 grid(unsigned(tiles), unsigned((nc + per - 1) / per));
-  k_dtheta<<<grid, kThreads, smem_bytes(), st>>>(d, s0, nc, ut, nt, per, xa, Ba, xb, Bb, dtheta);
+  int64_t rows = 0;
+  int n1max = 1;
+  for (int p = 0; p < d.P; ++p) {
+    const DevPath& q = d.path[p];
+    const int64_t tp = int64_t((q.c_in + kTU - 1) / kTU) * ((d.R * q.c_out + kTN - 1) / kTN);
+    rows += tp * nc * (2 * q.l1 + 1);
+    n1max = std::max(n1max, 2 * int(q.l1) + 1);
+  }
+  int64_t per = std::max<int64_t>(16, (rows + slots - 1) / slots);
+  auto ctas = [&](int64_t rp, int64_t* ymax) {
+    int64_t n = 0;
+    *ymax = 1;
+    for (int p = 0; p < d.P; ++p) {
+      const DevPath& q = d.path[p];
+      const int64_t tp = int64_t((q.c_in + kTU - 1) / kTU) * ((d.R * q.c_out + kTN - 1) / kTN);
+      const int64_t n1 = 2 * q.l1 + 1, nps = std::max<int64_t>(1, (rp + n1 - 1) / n1);
+      const int64_t y = (nc + nps - 1) / nps;
+      n += tp * y;
+      *ymax = std::max(*ymax, y);
+    }
+    return n;
+  };
+  int64_t ymax = 1;
+  while (ctas(per, &ymax) > slots && per < int64_t(nc) * n1max) per += per / 16 + 1;
+  ctas(per, &ymax);
+  const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(ymax));
+  k_dtheta<<<grid, kThreads, smem_bytes(), st>>>(d, s0, nc, ut, nt, int(std::min<int64_t>(per, 1 << 30)), xa, Ba, xb,
+                                                 Bb, dtheta);
   return cudaGetLastError();
 }
 
