@@ -1,9 +1,16 @@
 // Node-level contractions of the channel-wise operator family (see channelwise.h).
 //
-// Every kernel runs 32 x 8 thread blocks: x spans 32 consecutive channels (or
-// state columns), so each row of A / G / B is read or written as whole 128-byte
-// lines; y spans nodes of the chunk, grid-strided.  The grid holds about eight
-// blocks per SM.  Theta is a few KB and stays in L1.
+// Two forms of each map:
+//   * four channels per thread (every multiplicity a multiple of 4, Theta
+//     16-byte aligned): one thread per (node, group of 4 channels or state
+//     columns), rows of the block unrolled, state moved as float4 with
+//     streaming loads / stores;
+//   * one channel per thread otherwise: 32 x 8 thread blocks, x over 32
+//     consecutive channels (or state columns), y over nodes, grid-strided,
+//     about eight blocks per SM.
+// Either way a warp reads or writes each state row as whole 128-byte lines.
+// Theta is a few KB and stays in L1.  The Theta gradient reduces the node rows
+// of a block in shared memory and adds one partial per Theta entry and block.
 #include <cuda_runtime.h>
 
 #include <stdint.h>
