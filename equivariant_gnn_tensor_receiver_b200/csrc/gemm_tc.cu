@@ -490,17 +490,19 @@ cudaError_t split_elementwise(const float* v, int64_t n, float* hi, float* lo, c
   return cudaGetLastError();
 }
 
-// Theta of the paths of input block i1 as [c_in][K_x] with column kxoff(p) + k*c_out + w
-// (dx = B . Theta operand); optional TF32 split.
-__global__ void k_theta_x(const float* __restrict__ th, int64_t theta_off, int R, int c_in, int c_out, int kxoff,
-                          int Kx, float* __restrict__ hi, float* __restrict__ lo) {
-  const int64_t n = int64_t(R) * c_in * c_out;
+// Theta of each path as [c_in][K_x] of its input block, column kxoff(p) + k*c_out + w
+// (dx = B . Theta operand); optional TF32 split.  blockIdx.y = path of the list; the
+// blocks along x stride over its R c_in c_out entries.
+__global__ void k_theta_x_all(const float* __restrict__ th, const __grid_constant__ XPackList l,
+                              float* __restrict__ hi, float* __restrict__ lo) {
+  const XPackPath& q = l.p[blockIdx.y];
+  const int64_t n = int64_t(l.R) * q.c_in * q.c_out;
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
-    const int w = int(i % c_out);
-    const int64_t t = i / c_out;
-    const int u = int(t % c_in), k = int(t / c_in);
-    const float a = th[theta_off + i];  // Theta[p][k][u][w]
-    const int64_t o = int64_t(u) * Kx + kxoff + int64_t(k) * c_out + w;
+    const int w = int(i % q.c_out);
+    const int64_t t = i / q.c_out;
+    const int u = int(t % q.c_in), k = int(t / q.c_in);
+    const float a = th[q.theta_off + i];  // Theta[p][k][u][w]
+    const int64_t o = q.dst_off + int64_t(u) * q.Kx + q.kxoff + int64_t(k) * q.c_out + w;
     if (lo) {
       const float h = rn_tf32(a);
       hi[o] = h;
@@ -511,12 +513,13 @@ __global__ void k_theta_x(const float* __restrict__ th, int64_t theta_off, int R
   }
 }
 
-cudaError_t theta_x_pack(const float* th, int64_t theta_off, int R, int c_in, int c_out, int kxoff, int Kx, float* hi,
-                         float* lo, cudaStream_t st) {
-  const int64_t n = int64_t(R) * c_in * c_out;
-  if (n <= 0) return cudaSuccess;
-  const int blocks = int(std::min<int64_t>((n + 255) / 256, 148 * 8));
-  k_theta_x<<<blocks, 256, 0, st>>>(th, theta_off, R, c_in, c_out, kxoff, Kx, hi, lo);
+cudaError_t theta_x_pack_all(const float* th, const XPackList& l, float* hi, float* lo, cudaStream_t st) {
+  if (l.n <= 0 || l.n > kXPackMax) return l.n == 0 ? cudaSuccess : cudaErrorInvalidValue;
+  int64_t nmax = 0;
+  for (int i = 0; i < l.n; ++i) nmax = std::max<int64_t>(nmax, int64_t(l.R) * l.p[i].c_in * l.p[i].c_out);
+  if (nmax <= 0) return cudaSuccess;
+  const int bx = int(std::min<int64_t>((nmax + 255) / 256, std::max(1, 148 * 8 / l.n)));
+  k_theta_x_all<<<dim3(unsigned(bx), unsigned(l.n)), 256, 0, st>>>(th, l, hi, lo);
   return cudaGetLastError();
 }
 

@@ -25,9 +25,18 @@ cudaError_t split_transpose(const float* th, int K, int N, float* hi, float* lo,
 // hi = rn_tf32(v), lo = rn_tf32(v - hi) elementwise (lo null: plain copy)
 cudaError_t split_elementwise(const float* v, int64_t n, float* hi, float* lo, cudaStream_t st);
 
-// Theta[p] ([R][c_in][c_out]) into columns kxoff + k*c_out + w of a [c_in][Kx] matrix (split when lo != null)
-cudaError_t theta_x_pack(const float* th, int64_t theta_off, int R, int c_in, int c_out, int kxoff, int Kx, float* hi,
-                         float* lo, cudaStream_t st);
+// Theta[p] ([R][c_in][c_out]) of every listed path into columns kxoff + k*c_out + w of its [c_in][Kx]
+// matrix at dst_off (split when lo != null), all paths in one launch
+struct XPackPath {
+  int64_t theta_off, dst_off;
+  int c_in, c_out, kxoff, Kx;
+};
+constexpr int kXPackMax = 48;
+struct XPackList {
+  int n, R;
+  XPackPath p[kXPackMax];
+};
+cudaError_t theta_x_pack_all(const float* th, const XPackList& l, float* hi, float* lo, cudaStream_t st);
 
 // rows (node, m) x columns w of one feature block of nodes r0 : r0+nc -> dense [nc*n3][mul]
 cudaError_t pack_rows(const float* g, int dim, int off, int mul, int n3, int64_t r0, int nc, float* out,

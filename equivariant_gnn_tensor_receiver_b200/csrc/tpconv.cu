@@ -253,6 +253,14 @@ int64_t x_block_off(const DevPlan& d, int i1) {
   return o;
 }
 
+// kernel launches of prep_tc_theta
+int64_t tc_theta_launches(const DevPlan& d, bool needT, bool needN, bool needX) {
+  int64_t n = (needN ? 1 : 0) + (needX && d.P > 0 ? 1 : 0);
+  if (needT)
+    for (int i3 = 0; i3 < d.n_out; ++i3) n += first_path_of_out_block(d, i3) >= 0;
+  return n;
+}
+
 cudaError_t prep_tc_theta(const tpconv_plan* plan, const float* theta, float* region, int slot, bool needT,
                           bool needN, bool needX, TcTheta* o, cudaStream_t st) {
   const DevPlan& d = plan->dp;
@@ -272,13 +280,15 @@ cudaError_t prep_tc_theta(const tpconv_plan* plan, const float* theta, float* re
     o->N_lo = split ? b + 3 * tn : nullptr;
   }
   if (needX) {
+    static_assert(kXPackMax >= kMaxPaths, "one launch packs every path");
+    XPackList xl;
+    xl.n = d.P;
+    xl.R = d.R;
     for (int p = 0; p < d.P; ++p) {
       const DevPath& q = d.path[p];
-      const int64_t xo = x_block_off(d, q.i1);
-      if ((e = theta_x_pack(theta, q.theta_off, d.R, q.c_in, q.c_out, q.kxoff, d.Kx[q.i1], b + 4 * tn + xo,
-                            split ? b + 5 * tn + xo : nullptr, st)))
-        return e;
+      xl.p[p] = XPackPath{q.theta_off, x_block_off(d, q.i1), q.c_in, q.c_out, q.kxoff, d.Kx[q.i1]};
     }
+    if ((e = theta_x_pack_all(theta, xl, b + 4 * tn, split ? b + 5 * tn : nullptr, st))) return e;
     o->X_hi = b + 4 * tn;
     o->X_lo = split ? b + 5 * tn : nullptr;
   }
@@ -533,7 +543,7 @@ int tpconv_forward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t*
     if (prep_tc_theta(plan, theta, treg, 0, true, false, false, &tc, s)) return TPCONV_ERR_CUDA;
     thT_hi = tc.T_hi;
     thT_lo = tc.T_lo;
-    note(TPCONV_PHASE_OTHER, d.n_out);
+    note(TPCONV_PHASE_OTHER, tc_theta_launches(d, true, false, false));
   }
   for (int64_t r0 = 0; r0 < N; r0 += L.chunk_nodes) {
     const int nc = int(std::min<int64_t>(L.chunk_nodes, N - r0));
@@ -584,7 +594,7 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
   if (use_tc(plan)) {
     PhaseScope ps(TPCONV_PHASE_OTHER, s);
     if (prep_tc_theta(plan, theta, treg, 0, false, want_edge && E > 0, dx != nullptr, &tc, s)) return TPCONV_ERR_CUDA;
-    note(TPCONV_PHASE_OTHER, 1 + d.P);
+    note(TPCONV_PHASE_OTHER, tc_theta_launches(d, false, want_edge && E > 0, dx != nullptr));
     tcp = &tc;
   }
   if (want_edge && E > 0) {
@@ -673,7 +683,7 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
         return TPCONV_ERR_CUDA;
       tc1p = &tc1;
     }
-    note(TPCONV_PHASE_OTHER, (has_t ? 2 : 1) * (d.n_out + 1 + d.P));
+    note(TPCONV_PHASE_OTHER, (has_t ? 2 : 1) * tc_theta_launches(d, d_g != nullptr, wantR, d_x != nullptr));
   }
   // d_g = A1 . Theta + A0 . gg_theta
   if (d_g) {
