@@ -24,6 +24,7 @@ import json
 import os
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -68,6 +69,9 @@ def parse():
                     help="operator family: fully connected or channel-wise per-path weights")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--degree", type=float, default=None, help="mean degree of the sweep workload")
+    ap.add_argument("--clock-log", default=None,
+                    help="file for the nvidia-smi clock samples of the timed region ({rank} is replaced); "
+                         "default: a temporary file")
     ap.add_argument("--workspace-cap", type=int, default=None,
                     help="bytes of node-side state per receiver chunk (default: none; 8 GiB for capacity)")
     return ap.parse_args()
@@ -342,8 +346,8 @@ def run_ours(args):
     L.tpconv_profile_reset()
     L.tpconv_profile_enable(True)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    clk_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv") if os.path.isdir(
-        os.path.join(ROOT, "gpurun_out")) else f"/tmp/tpconv_clocks_{rank}.csv"
+    clk_path = args.clock_log.format(rank=rank) if args.clock_log else os.path.join(
+        tempfile.gettempdir(), f"tpconv_clocks_{os.getpid()}_{rank}.csv")
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(dev.index, clk_path) as clk:
@@ -437,6 +441,7 @@ def run_ours(args):
             "clocks": clk.summary(),
             "phases_ms": {k: round(v, 4) for k, v in phase_ms.items() if v > 0},
             "peak_mem_bytes": peak_mem, "workspace_bytes": ws_bytes, "resident_bytes_before_step": base_alloc,
+            "library_static_bytes": L.static_device_bytes(),
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -257,5 +257,15 @@ def tpconv_profile_read(phase: int):
     return ms.value, n.value
 
 
+STATIC_SCRATCH_BYTES = 64 << 20  # TPCONV_STATIC_SCRATCH_BYTES
+
+
+def static_device_bytes() -> int:
+    """Device memory the loaded library holds on every device by itself: the
+    fixed scratch array of ``tpconv_forward_static`` (resident whether or not
+    that entry point is called; not visible to torch's allocator statistics)."""
+    return STATIC_SCRATCH_BYTES
+
+
 def profile_all():
     return {name: tpconv_profile_read(i) for i, name in enumerate(PHASES)}

@@ -387,21 +387,25 @@ cudaError_t run(const float* A, int64_t lda, const float* B, const float* Blo, i
   if (SPLIT && !make_map(&tbl, Blo, N, K, ldb, BN)) return cudaErrorInvalidValue;
   if (!SPLIT) tbl = tb;
   using SM = TcSmem<BN>;
-  static bool attr_done[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SM::kBytes);
-    if (e) return e;
-    attr_done[dev] = true;
-  }
   dim3 grid(unsigned((M + kBM - 1) / kBM), unsigned((N + BN - 1) / BN));
   k_gemm_tc<BN, SPLIT><<<grid, 192, SM::kBytes, st>>>(ta, tb, tbl, M, N, K, out, accumulate);
   return cudaGetLastError();
 }
 
+template <int BN, bool SPLIT>
+cudaError_t set_smem() {
+  return cudaFuncSetAttribute(k_gemm_tc<BN, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcSmem<BN>::kBytes);
+}
+
 }  // namespace
+
+cudaError_t gemm_tc_init() {
+  cudaError_t e = cudaSuccess;
+  for (cudaError_t r : {set_smem<32, true>(), set_smem<64, true>(), set_smem<128, true>(), set_smem<256, true>(),
+                        set_smem<32, false>(), set_smem<64, false>(), set_smem<128, false>(), set_smem<256, false>()})
+    if (r != cudaSuccess && e == cudaSuccess) e = r;
+  return e;
+}
 
 bool gemm_tc_supported(const float* A, int64_t lda, const float* B, int64_t ldb, int M, int N, int K) {
   if (!encoder()) return false;

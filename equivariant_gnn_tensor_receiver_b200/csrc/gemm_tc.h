@@ -12,6 +12,9 @@ struct TcOut {
   int64_t rdiv, r_hi, r_lo, c_hi;
 };
 
+// Per-context set-up: the kernels' dynamic shared-memory limits.
+cudaError_t gemm_tc_init();
+
 // TMA / descriptor requirements: 16-byte aligned bases, row pitches a multiple of 4 floats.
 bool gemm_tc_supported(const float* A, int64_t lda, const float* B, int64_t ldb, int M, int N, int K);
 

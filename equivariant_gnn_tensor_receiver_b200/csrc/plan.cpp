@@ -493,7 +493,9 @@ int tpc::ws_layout(const tpconv_plan& p, int op, int64_t N, int64_t E, WsLayout*
   L->state_bytes = size_t(Nc) * size_t(per_node) * 4;
   off = align256(off + L->state_bytes);
   L->off_theta = off;
-  L->theta_bytes = align256(((p.theta_numel + 63) & ~size_t(63)) * 4 * 12);  // 2 Thetas x {T, N, X} x {hi, lo}
+  const bool tc = p.dp.family == TPCONV_FAMILY_FULL && (p.opt.gemm == TPCONV_GEMM_FP32 || p.opt.gemm == TPCONV_GEMM_TF32);
+  const int nreg = theta_region_count(op, tc, p.opt.gemm == TPCONV_GEMM_FP32);
+  L->theta_bytes = align256(((p.theta_numel + 63) & ~size_t(63)) * 4 * size_t(nreg));
   off = align256(off + L->theta_bytes);
   L->off_pack = off;
   L->pack_bytes = align256(size_t(Nc) * size_t(p.dp.dim_out) * 4);

@@ -9,8 +9,10 @@
 //   * a fixed-latency loop that must not call cudaMalloc / cudaFree, which can
 //     synchronise the device.
 // tpconv_forward_static serves them from a file-scope __device__ array of
-// TPCONV_STATIC_SCRATCH_BYTES.  Its address is looked up once per device with
-// cudaGetSymbolAddress; nothing here allocates.
+// TPCONV_STATIC_SCRATCH_BYTES.  Its device address is looked up with
+// cudaGetSymbolAddress on every call (a host-side query, no device work), so a
+// context that was reset and re-created never sees a stale address; nothing
+// here allocates.
 //
 // No part of the scratch has to start at zero: the forward writes every region
 // of its workspace (node state, tensor-core operands of Theta, packed output
@@ -21,29 +23,19 @@
 // serialised by the caller, e.g. by issuing them on one stream.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "../../include/tpconv.h"
 
 namespace {
 
 static __device__ __align__(256) unsigned char g_scratch[TPCONV_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_addr[kMaxDevices];
-
-// device address of g_scratch on the current device (looked up on first use)
+// device address of g_scratch in the current device's context.  The host-side
+// symbol g_scratch is only a handle: code on the host must never dereference it
+// or pass it to a kernel, only the address returned here.
 int scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TPCONV_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return TPCONV_ERR_CUDA;
-    g_addr[dev] = p;
-  }
-  *out = g_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return TPCONV_ERR_CUDA;
+  *out = p;
   return TPCONV_OK;
 }
 

@@ -41,16 +41,42 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-bool g_ready[kMaxDevices];
+unsigned long long g_ready_ctx[kMaxDevices];  // id of the context set up per device (0 = none)
 
-// Once per device: upload the real-CG table and raise the kernels' shared memory
-// limit.  The first call on a device synchronises it (cudaMemcpyToSymbol), so it
-// must not happen inside a stream capture.
+// Id of the current CUDA context (driver entry point, looked up once); 0 when
+// unavailable.  A device reset destroys the context and with it the constant
+// tables, so the set-up below is keyed on the context, not on the device.
+unsigned long long current_context_id() {
+  using GetCur = int (*)(void**);
+  using GetId = int (*)(void*, unsigned long long*);
+  static GetCur get_cur = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<GetCur>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+  });
+  void* ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_cur || !get_id || get_cur(&ctx) != 0 || !ctx || get_id(ctx, &id) != 0) return 0;
+  return id;
+}
+
+// Once per device context: upload the real-CG table and raise the kernels'
+// shared memory limit.  The first call in a context synchronises the device
+// (cudaMemcpyToSymbol), so it must not happen inside a stream capture.
 int ensure_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TPCONV_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (g_ready[dev]) return TPCONV_OK;
+  const unsigned long long ctx = current_context_id();
+  if (g_ready_ctx[dev] != 0 && (ctx == 0 || g_ready_ctx[dev] == ctx)) return TPCONV_OK;
   const float* t = cg_table_f32();
   if (!t) return TPCONV_ERR_INTERNAL;
   for (const TuInit& tu : tu_registry()) {
@@ -58,7 +84,9 @@ int ensure_device() {
     if (tu.smem && tu.smem(227 * 1024) != cudaSuccess) return TPCONV_ERR_CUDA;
   }
   if (dtheta_smem_init() != cudaSuccess) return TPCONV_ERR_CUDA;
-  g_ready[dev] = true;
+  if (gemm_tc_init() != cudaSuccess) return TPCONV_ERR_CUDA;
+  const unsigned long long now = current_context_id();  // the set-up above created the context if needed
+  g_ready_ctx[dev] = now ? now : ~0ull;
   return TPCONV_OK;
 }
 
@@ -261,25 +289,34 @@ int64_t tc_theta_launches(const DevPlan& d, bool needT, bool needN, bool needX) 
   return n;
 }
 
-cudaError_t prep_tc_theta(const tpconv_plan* plan, const float* theta, float* region, int slot, bool needT,
+cudaError_t prep_tc_theta(const tpconv_plan* plan, int op, const float* theta, float* region, int slot, bool needT,
                           bool needN, bool needX, TcTheta* o, cudaStream_t st) {
   const DevPlan& d = plan->dp;
   const size_t tn = (plan->theta_numel + 63) & ~size_t(63);
   const bool split = plan->opt.gemm == TPCONV_GEMM_FP32;
-  float* b = region + size_t(slot) * 6 * tn;
+  // slice (kind, half) of this slot; null when the operation reserves none
+  auto sl = [&](int kind, int half) -> float* {
+    const int i = theta_region(op, slot, kind, half, true, split);
+    return i < 0 ? nullptr : region + size_t(i) * tn;
+  };
   cudaError_t e;
   if (needT) {
-    if ((e = prep_theta_T(plan, theta, b, split ? b + tn : nullptr, st))) return e;
-    o->T_hi = b;
-    o->T_lo = split ? b + tn : nullptr;
+    float *hi = sl(kThetaT, 0), *lo = sl(kThetaT, 1);
+    if (!hi || (split && !lo)) return cudaErrorInvalidValue;
+    if ((e = prep_theta_T(plan, theta, hi, lo, st))) return e;
+    o->T_hi = hi;
+    o->T_lo = lo;
   }
   if (needN) {
-    if ((e = split_elementwise(theta, int64_t(plan->theta_numel), b + 2 * tn, split ? b + 3 * tn : nullptr, st)))
-      return e;
-    o->N_hi = b + 2 * tn;
-    o->N_lo = split ? b + 3 * tn : nullptr;
+    float *hi = sl(kThetaN, 0), *lo = sl(kThetaN, 1);
+    if (!hi || (split && !lo)) return cudaErrorInvalidValue;
+    if ((e = split_elementwise(theta, int64_t(plan->theta_numel), hi, lo, st))) return e;
+    o->N_hi = hi;
+    o->N_lo = lo;
   }
   if (needX) {
+    float *hi = sl(kThetaX, 0), *lo = sl(kThetaX, 1);
+    if (!hi || (split && !lo)) return cudaErrorInvalidValue;
     static_assert(kXPackMax >= kMaxPaths, "one launch packs every path");
     XPackList xl;
     xl.n = d.P;
@@ -288,9 +325,9 @@ cudaError_t prep_tc_theta(const tpconv_plan* plan, const float* theta, float* re
       const DevPath& q = d.path[p];
       xl.p[p] = XPackPath{q.theta_off, x_block_off(d, q.i1), q.c_in, q.c_out, q.kxoff, d.Kx[q.i1]};
     }
-    if ((e = theta_x_pack_all(theta, xl, b + 4 * tn, split ? b + 5 * tn : nullptr, st))) return e;
-    o->X_hi = b + 4 * tn;
-    o->X_lo = split ? b + 5 * tn : nullptr;
+    if ((e = theta_x_pack_all(theta, xl, hi, lo, st))) return e;
+    o->X_hi = hi;
+    o->X_lo = lo;
   }
   return cudaSuccess;
 }
@@ -540,7 +577,7 @@ int tpconv_forward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t*
   if (use_tc(plan)) {
     PhaseScope ps(TPCONV_PHASE_OTHER, s);
     TcTheta tc;
-    if (prep_tc_theta(plan, theta, treg, 0, true, false, false, &tc, s)) return TPCONV_ERR_CUDA;
+    if (prep_tc_theta(plan, TPCONV_OP_FORWARD, theta, treg, 0, true, false, false, &tc, s)) return TPCONV_ERR_CUDA;
     thT_hi = tc.T_hi;
     thT_lo = tc.T_lo;
     note(TPCONV_PHASE_OTHER, tc_theta_launches(d, true, false, false));
@@ -593,7 +630,7 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
   const TcTheta* tcp = nullptr;
   if (use_tc(plan)) {
     PhaseScope ps(TPCONV_PHASE_OTHER, s);
-    if (prep_tc_theta(plan, theta, treg, 0, false, want_edge && E > 0, dx != nullptr, &tc, s)) return TPCONV_ERR_CUDA;
+    if (prep_tc_theta(plan, TPCONV_OP_BACKWARD, theta, treg, 0, false, want_edge && E > 0, dx != nullptr, &tc, s)) return TPCONV_ERR_CUDA;
     note(TPCONV_PHASE_OTHER, tc_theta_launches(d, false, want_edge && E > 0, dx != nullptr));
     tcp = &tc;
   }
@@ -676,10 +713,10 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
   if (use_tc(plan)) {
     PhaseScope ps(TPCONV_PHASE_OTHER, s);
     const bool wantR = d_vec && E > 0;
-    if (prep_tc_theta(plan, theta, treg, 0, d_g != nullptr, wantR, d_x != nullptr, &tc0, s)) return TPCONV_ERR_CUDA;
+    if (prep_tc_theta(plan, TPCONV_OP_DOUBLE_BACKWARD, theta, treg, 0, d_g != nullptr, wantR, d_x != nullptr, &tc0, s)) return TPCONV_ERR_CUDA;
     tc0p = &tc0;
     if (has_t) {
-      if (prep_tc_theta(plan, gg_theta, treg, 1, d_g != nullptr, wantR, d_x != nullptr, &tc1, s))
+      if (prep_tc_theta(plan, TPCONV_OP_DOUBLE_BACKWARD, gg_theta, treg, 1, d_g != nullptr, wantR, d_x != nullptr, &tc1, s))
         return TPCONV_ERR_CUDA;
       tc1p = &tc1;
     }

@@ -58,6 +58,9 @@ extern "C" {
 #endif
 
 /* status codes */
+/* Device set-up (constant tables, kernel attributes) is done once per CUDA
+ * context on the first call that needs it; a context destroyed by
+ * cudaDeviceReset is set up again on the next call. */
 #define TPCONV_OK 0
 #define TPCONV_ERR_INVALID_ARG 1        /* null/negative/misaligned argument   */
 #define TPCONV_ERR_BAD_IRREPS 2         /* irreps string does not parse         */
@@ -168,7 +171,10 @@ int tpconv_graph_transpose(const tpconv_plan* plan, int64_t N, int64_t E, const 
 
 /*
  * Forward (device, async): out[N][dim_out] from x[N][dim_in], theta[theta_numel]
- * and the receiver CSR graph with edge vectors.
+ * and the receiver CSR graph with edge vectors.  The operator of "Sobek"
+ * (arXiv 2607.18074), abstract, in the streaming form the abstract describes:
+ * a receiver-sorted edge stream accumulates A[r, k, p, u, m3] and a node-level
+ * contraction with Theta mixes it (formula at the top of this file).
  */
 int tpconv_forward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t* rowptr,
                    const int32_t* col, const float* edge_vec, const float* x, const float* theta,
@@ -187,13 +193,20 @@ int tpconv_forward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t*
  * zero.
  *   Returns TPCONV_ERR_WORKSPACE_TOO_SMALL, before any device work, when
  *   tpconv_workspace_size(plan, TPCONV_OP_FORWARD, N, E) exceeds
- *   TPCONV_STATIC_SCRATCH_BYTES; a plan created with a smaller workspace_cap
- *   (node chunks) fits.
+ *   TPCONV_STATIC_SCRATCH_BYTES.  The forward workspace is the node state of
+ *   one receiver chunk (bounded by workspace_cap) plus a Theta region that no
+ *   cap shrinks: 2 x theta_numel floats with GEMM_FP32, 1 x with GEMM_TF32,
+ *   none with GEMM_SIMT or the CHANNELWISE family.  A plan whose Theta region
+ *   alone approaches the limit (e.g. 128x{0e,1o,2e,3o} with GEMM_FP32, 24 MB)
+ *   fits only with a small cap; tpconv_workspace_size says which.
  *   Calls share the array: calls that overlap in time (other streams, other
  *   host threads) race on it and must be serialised by the caller.
  *   The first call on a device also performs the library's one-time device
- *   set-up (constant tables, kernel attributes, the array's address), which
- *   synchronises the device: make it before any stream capture.
+ *   set-up (constant tables, kernel attributes), which synchronises the
+ *   device: make it before any stream capture.  The array's device address is
+ *   looked up on every call (cudaGetSymbolAddress, a host-side query).
+ *   Every device on which the library is loaded holds the array until the
+ *   process exits, whether or not this entry point is called.
  */
 #define TPCONV_STATIC_SCRATCH_BYTES (64u << 20) /* 64 MiB */
 int tpconv_forward_static(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t* rowptr,
@@ -201,7 +214,11 @@ int tpconv_forward_static(const tpconv_plan* plan, int64_t N, int64_t E, const i
                           float* out, void* stream);
 
 /*
- * Backward (device, async) for the cotangent g[N][dim_out] of out.
+ * Backward (device, async) for the cotangent g[N][dim_out] of out: the first
+ * differentiation order of the operator ("Sobek", arXiv 2607.18074, abstract:
+ * the streaming schedule extends through backward), run as a sender-sorted
+ * stream into sender-side state B plus node contractions (dx = B . Theta,
+ * dtheta = x^T B) and a receiver-sorted adjoint stream (dvec, dY, db).
  *   dx[N][dim_in], dtheta[theta_numel], dvec[E][3] (CSR order): optional.
  *   dY[E][n_sh], db[E][R]: optional per-edge adjoints of the spherical
  *   harmonics and radial basis (CSR order).
@@ -215,7 +232,8 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
                     float* dY, float* db, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * Double backward (device, async).  With Psi = <gg_x, dx> + <gg_vec, dvec> +
+ * Double backward (device, async): the second differentiation order the
+ * abstract of "Sobek" (arXiv 2607.18074) names.  With Psi = <gg_x, dx> + <gg_vec, dvec> +
  * <gg_theta, dtheta> for the first-order gradients of <g, out>, returns
  * d_g = dPsi/dg [N][dim_out], d_x = dPsi/dx, d_vec = dPsi/dedge_vec [E][3] and
  * d_theta = dPsi/dtheta.  Each cotangent gg_* may be NULL (= zero); each

@@ -119,3 +119,28 @@ def test_bf16_mixing_is_reported_unsupported(T):
     with pytest.raises(T.TPConvError) as e:
         T.Plan("8x0e+8x1o", 2, "8x0e+8x1o", 4, gemm="bf16")
     assert e.value.status == 3  # TPCONV_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("gemm,per_op", [("fp32", (2, 4, 12)), ("tf32", (1, 2, 6)), ("simt", (0, 0, 0))])
+def test_theta_region_sized_per_operation(T, gemm, per_op):
+    """The repacked Theta operands of the tensor-core contractions take what each
+    operation uses: forward Theta^T (hi, lo), backward the elementwise split and
+    the dx packing, double backward all three for Theta and gg_Theta; none
+    without tensor cores.  The wide plan's forward fits the fixed 64 MiB scratch
+    of the allocation-free forward only with a node cap."""
+    c = W.CONFIGS["wide"]
+    L = T._lib
+
+    def size(cap):
+        p = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], gemm=gemm, workspace_cap=cap)
+        return p, [L.tpconv_workspace_size(p, op, 8192, 262_144) for op in (0, 1, 2)]
+
+    plan, a = size(1)           # one node per chunk: the Theta region dominates
+    tn = (plan.theta_numel + 63) // 64 * 64 * 4
+    for got, k in zip(a, per_op):
+        assert k * tn <= got <= k * tn + (1 << 20), (got, k * tn)
+    _, b = size(0)
+    state = 4 * 8192 * 101_376  # A floats per node of the wide layer
+    assert b[0] >= state + per_op[0] * tn
+    if gemm == "fp32":
+        assert a[0] <= L.STATIC_SCRATCH_BYTES < b[0]
