@@ -6,14 +6,18 @@ mace-like layer (4096 atoms in a periodic box at 0.1 atoms/A^3, all pairs within
 5 A, 64x0e+64x1o+64x2e -> same, SH l<=3, R=8 Bessel radial basis): sender-sorted
 graph view, forward, backward (dx, dTheta, dvec) and double backward in the
 force-training shape (gg_x, gg_vec given, gg_Theta = 0) -> d_g, d_x, d_vec,
-d_Theta.  The headline value is edges per second of that step.
+d_Theta.  The headline value is edges per second of that step; the same line
+carries edges/s of the forward alone, of forward + backward and of the double
+backward alone.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --suite [--steps K]    # one line per workload of the metric
 
 N > 1 runs under torch.distributed.run: every rank processes its own graph
 (seed = rank) with no collective on the data path (weak scaling); the step time
-is the max over ranks.  --impl reference times the CPU oracle on a bounded
-sample of the same workload (the pages ship no runnable reference).
+is the max over ranks.  --impl reference times the CPU oracle (the
+conventional schedule) on bounded samples of the same workload, one process
+per host core (the pages ship no runnable reference).
 """
 
 from __future__ import annotations
@@ -68,6 +72,13 @@ def parse():
     ap.add_argument("--family", default="full", choices=["full", "channelwise"],
                     help="operator family: fully connected or channel-wise per-path weights")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--suite", action="store_true",
+                    help="one JSON line per workload (tiny, mace, sweep d=25/100/400, wide fp32/tf32): "
+                         "fwd, fwd+bwd and double-bwd edges/s, peak memory, roofline of the dominant kernel")
+    ap.add_argument("--suite-configs", default="tiny,mace,sweep25,sweep100,sweep400,wide_fp32,wide_tf32",
+                    help="comma-separated suite entries (also: capacity)")
+    ap.add_argument("--oracle-procs", type=int, default=0,
+                    help="processes of the CPU oracle baseline (default: the host cores, at most 32)")
     ap.add_argument("--degree", type=float, default=None, help="mean degree of the sweep workload")
     ap.add_argument("--clock-log", default=None,
                     help="file for the nvidia-smi clock samples of the timed region ({rank} is replaced); "
@@ -178,13 +189,11 @@ class ClockSampler:
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "reasons": reasons, "samples": len(rows)}
 
 
-def cpu_cores():
+def host_cores():
     try:
-        from threadpoolctl import threadpool_info
-        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
-    except Exception:
-        n = 1
-    return int(n)
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 def theta_segments(paths, R, family):
@@ -227,6 +236,69 @@ def oracle_sample(cfg, graph, n_recv, seed=100, family="full"):
     return step, e1
 
 
+def _oracle_proc(cfg, family, r0, n_recv, warmup, steps, ready, start, out):
+    """One process of the parallel oracle baseline: the oracle step on the
+    edges of receivers r0 .. r0+n_recv-1 (single-threaded BLAS), `warmup`
+    untimed steps, then `steps` timed ones once every process is ready."""
+    graph = W.graph_for(cfg, 0)
+    rowptr, col, vec = graph
+    # the sample: receivers r0.. renumbered to 0.. (their senders keep their own rows)
+    e0, e1 = int(rowptr[r0]), int(rowptr[r0 + n_recv])
+    rp = np.asarray(rowptr[r0:r0 + n_recv + 1], dtype=np.int64) - e0
+    sub = (rp, np.asarray(col[e0:e1]), vec[e0:e1])
+    step, e = oracle_sample(cfg, sub, n_recv, seed=100 + r0, family=family)
+    for _ in range(warmup):
+        step()
+    ready.put(os.getpid())
+    start.wait()
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        step()
+        times.append(time.perf_counter() - t0)
+    out.put((e, times))
+
+
+def parallel_oracle(cfg, family, procs, n_recv, warmup, steps):
+    """The CPU oracle (fp64 numpy, conventional schedule) timed on `procs`
+    processes at once, each on its own block of n_recv receivers of the
+    workload's graph.  Processes start with 'spawn' (never forked from a
+    process that has used the GPU) and run with one BLAS thread each, so
+    `procs` is the number of host cores busy.  Returns edges/s of all processes
+    together over the slowest process's time, per step."""
+    import multiprocessing as mp
+    env = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+    for k in env:
+        os.environ[k] = "1"
+    try:
+        ctx = mp.get_context("spawn")
+        ready, out, start = ctx.Queue(), ctx.Queue(), ctx.Event()
+        ps = [ctx.Process(target=_oracle_proc, args=(cfg, family, i * n_recv, n_recv, warmup, steps, ready, start, out))
+              for i in range(procs)]
+        for p in ps:
+            p.start()
+        for _ in ps:
+            ready.get(timeout=900)
+        start.set()
+        res = [out.get(timeout=3600) for _ in ps]
+        for p in ps:
+            p.join()
+    finally:
+        for k, v in env.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+    edges = sum(e for e, _ in res)
+    per_step = [max(t[i] for _, t in res) for i in range(steps)]
+    dt = sum(per_step) / steps
+    return {"value": edges / dt, "unit": "edges/s", "cores": procs, "kind": "oracle", "ms_per_step": dt * 1e3,
+            "edges_per_step": edges,
+            "sample": f"fp64 numpy oracle step (fwd + bwd + double bwd, conventional schedule) on {procs} "
+                      f"processes x {n_recv} receivers ({edges} edges per step, one BLAS thread each), "
+                      f"{steps} timed steps"}
+
+
 def reduce_over_ranks(v, op, world, device):
     """Max or sum of a per-rank scalar over the default process group (any
     backend: nccl with a CUDA device, gloo with the CPU); identity at world 1."""
@@ -251,25 +323,194 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    graph = W.graph_for(args.config, 0)
-    n_recv = 8
-    step, e = oracle_sample(args.config, graph, n_recv, family=args.family)
-    for _ in range(args.warmup):
-        step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
-    dt = (time.perf_counter() - t0) / args.steps
-    v = e / dt
-    cores = cpu_cores()
+    procs = args.oracle_procs or min(32, host_cores())
+    r = parallel_oracle(args.config, args.family, procs, 4, max(1, min(args.warmup, 1)), args.steps)
+    v = r["value"]
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "edges/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload(args), "sample": f"edges of the first {n_recv} receivers ({e} edges)"},
-            "cpu_baseline": {"value": v, "unit": "edges/s", "cores": cores, "kind": "oracle",
-                             "sample": f"fp64 numpy oracle, conventional schedule, {e} edges per step"},
+            "config": {"workload": workload(args), "sample": r["sample"]},
+            "cpu_baseline": {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")},
             "e2e": {"value": v, "unit": "edges/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+class Work:
+    """One workload resident on the device: plan, inputs, outputs, workspaces
+    and the library calls of one step (all arithmetic in the CUDA library)."""
+
+    def __init__(self, T, L, config, graph, gemm, family, cap, dev, seed=0):
+        import torch
+        c = W.CONFIGS[config]
+        self.L, self.dev = L, dev
+        rowptr, col, vec = graph
+        self.N, self.E = N, E = len(rowptr) - 1, len(col)
+        self.plan = plan = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], radial=c["radial"],
+                                  radial_params=c["radial_params"], gemm=gemm, workspace_cap=cap, family=family)
+        f32 = torch.float32
+        pin = lambda a, dt=f32: torch.as_tensor(np.ascontiguousarray(a), dtype=dt).pin_memory()
+        self.host = {
+            "rowptr": pin(rowptr, torch.int32), "col": pin(col, torch.int32), "vec": pin(vec),
+            "x": pin(W.normal((N, plan.dim_in), 10 + seed)),
+            "theta": pin(W.theta(theta_segments(plan.paths, plan.R, family), 11 + seed)),
+            "g": pin(W.normal((N, plan.dim_out), 12 + seed)),
+            "gg_x": pin(W.normal((N, plan.dim_in), 13 + seed)),
+            "gg_vec": pin(W.normal((E, 3), 14 + seed)),
+        }
+        self.d = {k: v.to(dev) for k, v in self.host.items()}
+        self.outs = {
+            "out": torch.empty(N, plan.dim_out, device=dev), "dx": torch.empty(N, plan.dim_in, device=dev),
+            "dtheta": torch.empty(plan.theta_numel, device=dev), "dvec": torch.empty(E, 3, device=dev),
+            "d_g": torch.empty(N, plan.dim_out, device=dev), "d_x": torch.empty(N, plan.dim_in, device=dev),
+            "d_vec": torch.empty(E, 3, device=dev), "d_theta": torch.empty(plan.theta_numel, device=dev),
+        }
+        self.perm = torch.empty(max(E, 1), dtype=torch.int32, device=dev)
+        self.s_rowptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
+        self.s_recv = torch.empty(max(E, 1), dtype=torch.int32, device=dev)
+        self.ws = {op: T.workspace(plan, op, N, E, dev) for op in (L.OP_FORWARD, L.OP_BACKWARD,
+                                                                   L.OP_DOUBLE_BACKWARD, L.OP_TRANSPOSE)}
+        self.ws_bytes = sum(w.numel() for w in self.ws.values())
+
+    def transpose(self, src=None):
+        src, L = src or self.d, self.L
+        L.tpconv_graph_transpose(self.plan, self.N, self.E, src["rowptr"], src["col"], self.perm, self.s_rowptr,
+                                 self.s_recv, self.ws[L.OP_TRANSPOSE])
+
+    def fwd(self, src=None):
+        src, L, o = src or self.d, self.L, self.outs
+        L.tpconv_forward(self.plan, self.N, self.E, src["rowptr"], src["col"], src["vec"], src["x"], src["theta"],
+                         o["out"], self.ws[L.OP_FORWARD])
+
+    def bwd(self, src=None):
+        src, L, o = src or self.d, self.L, self.outs
+        L.tpconv_backward(self.plan, self.N, self.E, src["rowptr"], src["col"], self.perm, self.s_rowptr,
+                          self.s_recv, src["vec"], src["x"], src["theta"], src["g"], o["dx"], o["dtheta"], o["dvec"],
+                          None, None, self.ws[L.OP_BACKWARD])
+
+    def dbl(self, src=None):
+        src, L, o = src or self.d, self.L, self.outs
+        L.tpconv_double_backward(self.plan, self.N, self.E, src["rowptr"], src["col"], self.perm, self.s_rowptr,
+                                 self.s_recv, src["vec"], src["x"], src["theta"], src["g"], src["gg_x"],
+                                 src["gg_vec"], None, o["d_g"], o["d_x"], o["d_vec"], o["d_theta"],
+                                 self.ws[L.OP_DOUBLE_BACKWARD])
+
+    def step(self, src=None):
+        self.transpose(src)
+        self.fwd(src)
+        self.bwd(src)
+        self.dbl(src)
+
+
+def time_ms(fn, steps, flush):
+    """Mean device time (CUDA events on the current stream) of fn over `steps`
+    calls, L2 flushed (a buffer of twice its size zeroed) before each, outside
+    the events."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for a, b in evs:
+        flush.zero_()
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs) / steps
+
+
+def per_direction(work, steps, flush):
+    """edges/s of the forward alone, forward + backward (dx, dTheta, dvec; the
+    sender-sorted view is built once per graph, outside), and the double
+    backward alone (gg_x, gg_vec)."""
+    work.transpose()
+    t_f = time_ms(work.fwd, steps, flush)
+    t_fb = time_ms(lambda: (work.fwd(), work.bwd()), steps, flush)
+    t_d = time_ms(work.dbl, steps, flush)
+    E = work.E
+    return {"fwd_edges_per_s": E / (t_f * 1e-3), "fwd_bwd_edges_per_s": E / (t_fb * 1e-3),
+            "dbl_edges_per_s": E / (t_d * 1e-3), "fwd_ms": t_f, "fwd_bwd_ms": t_fb, "dbl_ms": t_d}
+
+
+def roofline(T, plan, prof_ms, E):
+    """FP32-ALU roofline of the dominant phase (algorithmic FMAs, see work_model)."""
+    peaks, peak_src = measured_peaks()
+    wm = work_model(T, plan)
+    dom = max(prof_ms, key=lambda k: prof_ms[k])
+    roof = {"phase": dom, "bound": None, "achieved": None, "peak": None, "unit": None, "frac": None,
+            "traffic": None}
+    sm_max = peaks.get("sm_max_mhz", 1965.0)
+    if dom in wm:
+        flops = 2.0 * wm[dom] * E
+        ach = flops / (prof_ms[dom] * 1e-3) / 1e12
+        peak = N_SM * FP32_LANES_PER_SM * 2 * sm_max * 1e6 / 1e12
+        roof.update(bound="alu", achieved=ach, peak=peak, unit="TFLOP/s", frac=ach / peak,
+                    peak_source=f"148 SM x 128 FP32 lanes x 2 x {sm_max:.0f} MHz (max clock, {peak_src} file)",
+                    work=f"{wm[dom]} algorithmic FMA per edge x {E} edges")
+    try:
+        with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+            tr = json.load(f).get(dom)
+        if tr and tr.get("sources_sha256") == sources_digest(tr["sources"]):
+            roof["traffic"] = tr["dram_bytes_per_launch"]
+            roof["traffic_kernel"] = tr["kernel"]
+    except (OSError, ValueError):
+        pass
+    return roof
+
+
+SUITE = {
+    # entry: (config, degree, gemm)
+    "tiny": ("tiny", None, "fp32"),
+    "mace": ("mace", None, "fp32"),
+    "sweep25": ("sweep", 25, "fp32"),
+    "sweep100": ("sweep", 100, "fp32"),
+    "sweep400": ("sweep", 400, "fp32"),
+    "wide_fp32": ("wide", None, "fp32"),
+    "wide_tf32": ("wide", None, "tf32"),
+    "capacity": ("capacity", None, "fp32"),
+}
+
+
+def run_suite(args):
+    """One JSON line per workload: edges/s of fwd, fwd+bwd and the double
+    backward, peak allocated memory (total and workspace), and the FP32-ALU
+    roofline fraction of the dominant edge-stream kernel of the full step."""
+    import torch
+
+    import equivariant_gnn_tensor_receiver_b200 as T
+    from equivariant_gnn_tensor_receiver_b200 import _lib as L
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    for name in args.suite_configs.split(","):
+        cfg, degree, gemm = SUITE[name]
+        cap = 8 << 30 if cfg == "capacity" else 0
+        steps = 2 if cfg == "capacity" else args.steps
+        graph = W.graph_for(cfg, 0, degree)
+        torch.cuda.empty_cache()
+        torch.cuda.reset_peak_memory_stats(dev)
+        base = torch.cuda.memory_allocated(dev)
+        w = Work(T, L, cfg, graph, gemm, args.family, cap, dev)
+        for _ in range(max(1, min(args.warmup, 3))):
+            w.step()
+        torch.cuda.synchronize()
+        L.tpconv_profile_reset()
+        L.tpconv_profile_enable(True)
+        t_step = time_ms(w.step, steps, flush)
+        L.tpconv_profile_enable(False)
+        prof_ms = {k: ms / steps for k, (ms, _) in L.profile_all().items()}
+        pd = per_direction(w, steps, flush)
+        peak = torch.cuda.max_memory_allocated(dev) - base
+        inputs = sum(v.numel() * v.element_size() for v in w.d.values())
+        outputs = sum(v.numel() * v.element_size() for v in w.outs.values())
+        line = {"suite": name, "workload": WORKLOADS[cfg].format(d=degree or 25), "gemm": gemm,
+                "family": args.family, "nodes": w.N, "edges": w.E, "steps": steps,
+                **{k: v for k, v in pd.items()},
+                "step_edges_per_s": w.E / (t_step * 1e-3), "step_ms": t_step,
+                "peak_mem_bytes": peak, "workspace_bytes": w.ws_bytes, "inputs_bytes": inputs,
+                "outputs_bytes": outputs, "roofline": roofline(T, w.plan, prof_ms, w.E),
+                "phases_ms": {k: round(v, 4) for k, v in prof_ms.items() if v > 0}}
+        print(json.dumps(line), flush=True)
+        del w
+        torch.cuda.synchronize()
 
 
 def run_ours(args):
@@ -287,48 +528,15 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
-    c = W.CONFIGS[args.config]
-    rowptr, col, vec = W.graph_for(args.config, rank, args.degree)
+    graph = W.graph_for(args.config, rank, args.degree)
+    rowptr, col, vec = graph
     N, E = len(rowptr) - 1, len(col)
     cap = args.workspace_cap if args.workspace_cap is not None else (8 << 30 if args.config == "capacity" else 0)
-    plan = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], radial=c["radial"],
-                  radial_params=c["radial_params"], gemm=args.gemm, workspace_cap=cap, family=args.family)
-    f32 = torch.float32
-    pin = lambda a, dt=f32: torch.as_tensor(np.ascontiguousarray(a), dtype=dt).pin_memory()
-    host = {
-        "rowptr": pin(rowptr, torch.int32), "col": pin(col, torch.int32), "vec": pin(vec),
-        "x": pin(W.normal((N, plan.dim_in), 10 + rank)),
-        "theta": pin(W.theta(theta_segments(plan.paths, plan.R, args.family), 11 + rank)),
-        "g": pin(W.normal((N, plan.dim_out), 12 + rank)),
-        "gg_x": pin(W.normal((N, plan.dim_in), 13 + rank)),
-        "gg_vec": pin(W.normal((E, 3), 14 + rank)),
-    }
-    d = {k: v.to(dev) for k, v in host.items()}
-    outs = {
-        "out": torch.empty(N, plan.dim_out, device=dev), "dx": torch.empty(N, plan.dim_in, device=dev),
-        "dtheta": torch.empty(plan.theta_numel, device=dev), "dvec": torch.empty(E, 3, device=dev),
-        "d_g": torch.empty(N, plan.dim_out, device=dev), "d_x": torch.empty(N, plan.dim_in, device=dev),
-        "d_vec": torch.empty(E, 3, device=dev), "d_theta": torch.empty(plan.theta_numel, device=dev),
-    }
+    work = Work(T, L, args.config, graph, args.gemm, args.family, cap, dev, seed=rank)
+    plan, host, d, outs, ws_bytes = work.plan, work.host, work.d, work.outs, work.ws_bytes
     hout = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in outs.items()}
-    perm = torch.empty(E, dtype=torch.int32, device=dev)
-    s_rowptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
-    s_recv = torch.empty(E, dtype=torch.int32, device=dev)
-    ws = {op: T.workspace(plan, op, N, E, dev) for op in (L.OP_FORWARD, L.OP_BACKWARD, L.OP_DOUBLE_BACKWARD,
-                                                          L.OP_TRANSPOSE)}
-    ws_bytes = sum(w.numel() for w in ws.values())
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
-
-    def step(src):
-        L.tpconv_graph_transpose(plan, N, E, src["rowptr"], src["col"], perm, s_rowptr, s_recv, ws[L.OP_TRANSPOSE])
-        L.tpconv_forward(plan, N, E, src["rowptr"], src["col"], src["vec"], src["x"], src["theta"], outs["out"],
-                         ws[L.OP_FORWARD])
-        L.tpconv_backward(plan, N, E, src["rowptr"], src["col"], perm, s_rowptr, s_recv, src["vec"], src["x"],
-                          src["theta"], src["g"], outs["dx"], outs["dtheta"], outs["dvec"], None, None,
-                          ws[L.OP_BACKWARD])
-        L.tpconv_double_backward(plan, N, E, src["rowptr"], src["col"], perm, s_rowptr, s_recv, src["vec"],
-                                 src["x"], src["theta"], src["g"], src["gg_x"], src["gg_vec"], None, outs["d_g"],
-                                 outs["d_x"], outs["d_vec"], outs["d_theta"], ws[L.OP_DOUBLE_BACKWARD])
+    step = work.step
 
     def barrier():
         if world > 1:
@@ -386,42 +594,21 @@ def run_ours(args):
     e2e_ms = allmax(sum(e2e) / len(e2e))
 
     # roofline of the dominant phase
-    peaks, peak_src = measured_peaks()
-    wm = work_model(T, plan)
     phase_ms = {k: ms / args.steps for k, (ms, _) in prof.items()}
-    dom = max(phase_ms, key=lambda k: phase_ms[k])
-    roof = {"phase": dom, "bound": None, "achieved": None, "peak": None, "unit": None, "frac": None,
-            "traffic": None}
-    sm_max = peaks.get("sm_max_mhz", 1965.0)
-    if dom in wm:
-        flops = 2.0 * wm[dom] * E
-        ach = flops / (phase_ms[dom] * 1e-3) / 1e12
-        peak = N_SM * FP32_LANES_PER_SM * 2 * sm_max * 1e6 / 1e12
-        roof.update(bound="alu", achieved=ach, peak=peak, unit="TFLOP/s", frac=ach / peak,
-                    peak_source=f"148 SM x 128 FP32 lanes x 2 x {sm_max:.0f} MHz (max clock, {peak_src} file)",
-                    work=f"{wm[dom]} algorithmic FMA per edge x {E} edges")
-    try:
-        with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
-            tr = json.load(f).get(dom)
-        if tr and tr.get("sources_sha256") == sources_digest(tr["sources"]):
-            roof["traffic"] = tr["dram_bytes_per_launch"]
-            roof["traffic_kernel"] = tr["kernel"]
-    except (OSError, ValueError):
-        pass
+    roof = roofline(T, plan, phase_ms, E)
 
+    per_dir = per_direction(work, args.steps, flush)
+    for k in ("fwd_ms", "fwd_bwd_ms", "dbl_ms"):  # slowest rank; every rank takes the same steps
+        per_dir[k] = allmax(per_dir[k])
+    E_all = allsum(float(E))
+    per_dir.update(fwd_edges_per_s=E_all / (per_dir["fwd_ms"] * 1e-3),
+                   fwd_bwd_edges_per_s=E_all / (per_dir["fwd_bwd_ms"] * 1e-3),
+                   dbl_edges_per_s=E_all / (per_dir["dbl_ms"] * 1e-3))
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        stepc, ec = oracle_sample(args.config, (rowptr, col, vec), 4, family=args.family)
-        stepc()
-        t0 = time.perf_counter()
-        reps = 0
-        while time.perf_counter() - t0 < 10.0 or reps < 1:
-            stepc()
-            reps += 1
-        dt = (time.perf_counter() - t0) / reps
-        cpu = {"value": ec / dt, "unit": "edges/s", "cores": cpu_cores(), "kind": "oracle",
-               "sample": f"fp64 numpy oracle step (fwd+bwd+double bwd) on the {ec} edges of 4 receivers, "
-                         f"{reps} reps"}
+        procs = args.oracle_procs or min(32, host_cores())
+        r = parallel_oracle(args.config, args.family, procs, 4, 1, 2)
+        cpu = {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")}
 
     if rank == 0:
         line = {
@@ -439,6 +626,7 @@ def run_ours(args):
             "roofline": roof,
             "cpu_baseline": cpu,
             "clocks": clk.summary(),
+            "per_direction": per_dir,
             "phases_ms": {k: round(v, 4) for k, v in phase_ms.items() if v > 0},
             "peak_mem_bytes": peak_mem, "workspace_bytes": ws_bytes, "resident_bytes_before_step": base_alloc,
             "library_static_bytes": L.static_device_bytes(),
@@ -453,6 +641,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.suite:
+        run_suite(args)
     else:
         run_ours(args)
 

@@ -60,6 +60,8 @@ _EXPORTS = {
     "tpconv_forward_static": (ctypes.c_int, [_P, _I64, _I64] + [_P] * 6 + [_P]),
     "tpconv_backward": (ctypes.c_int, [_P, _I64, _I64] + [_P] * 14 + [_P, ctypes.c_size_t, _P]),
     "tpconv_double_backward": (ctypes.c_int, [_P, _I64, _I64] + [_P] * 16 + [_P, ctypes.c_size_t, _P]),
+    "tpconv_get_device_status": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int)]),
+    "tpconv_set_wait_limit": (ctypes.c_int, [ctypes.c_uint64]),
     "tpconv_profile_enable": (ctypes.c_int, [ctypes.c_int]),
     "tpconv_profile_reset": (ctypes.c_int, []),
     "tpconv_profile_read": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_double),
@@ -239,6 +241,23 @@ def tpconv_double_backward(plan, N, E, rowptr, col, perm, s_rowptr, s_recv, edge
                                         _ptr(gg_vec, f32), _ptr(gg_theta, f32), _ptr(d_g, f32),
                                         _ptr(d_x, f32), _ptr(d_vec, f32), _ptr(d_theta, f32), w, wb,
                                         _stream(stream)))
+
+
+TPCONV_ERR_TIMEOUT = 7
+
+
+def tpconv_get_device_status(plan, stream=None) -> int:
+    """Synchronises the stream; TPCONV_ERR_TIMEOUT if a bounded device wait of
+    the tensor-core kernels expired since the last query (the record is
+    cleared), else TPCONV_OK."""
+    st = ctypes.c_int()
+    _check("tpconv_get_device_status", lib().tpconv_get_device_status(plan.handle, _stream(stream), ctypes.byref(st)))
+    return st.value
+
+
+def tpconv_set_wait_limit(ns: int):
+    """Limit (ns) of the tensor-core kernels' device waits for later calls; 0 = default (2 s)."""
+    _check("tpconv_set_wait_limit", lib().tpconv_set_wait_limit(int(ns)))
 
 
 def tpconv_profile_enable(on: bool = True):

@@ -27,7 +27,8 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-lineinfo", "-O3", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
                      "-Xptxas", "-v", f"-I{os.path.join(ROOT, 'include')}"]
-CXX_FLAGS = ["-O2", "-fPIC", "-std=c++17", f"-I{os.path.join(ROOT, 'include')}"]
+CUDA_HOME = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+CXX_FLAGS = ["-O2", "-fPIC", "-std=c++17", f"-I{os.path.join(ROOT, 'include')}", f"-I{os.path.join(CUDA_HOME, 'include')}"]
 
 
 def _cu_sources():

@@ -23,8 +23,9 @@
 // 128-byte swizzle) into a ring of shared-memory stages; warp 1 owns the TMEM
 // accumulator (128 lanes x BN fp32 columns) and issues the MMAs from one thread;
 // warps 2-5 split A (3xTF32) and run the epilogue (tcgen05.ld -> global).
-// Every wait is bounded; on expiry the kernel records an error code, stops
-// issuing work, waits (bounded) for its own loads, frees TMEM and returns.
+// Every wait on the pipeline is bounded by the call's wait limit; on expiry the
+// kernel records an error code and stops issuing work; before it exits it waits
+// (bounded by a fixed limit) for its own loads and MMAs, then frees TMEM.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -34,6 +35,7 @@
 #include <mutex>
 
 #include "gemm_tc.h"
+#include "tc_common.cuh"
 
 namespace tpc {
 
@@ -41,108 +43,15 @@ __device__ int g_tc_error;  // first error code recorded by a tensor-core GEMM (
 
 namespace {
 
+using namespace tc;
+
 constexpr int kBM = 128, kBK = 32;  // rows per CTA, fp32 K per stage (128 bytes)
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits give up after 2 s
 
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// bounded wait; returns false (and records `code`) when the limit expires
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, int code) {
-  if (mbar_try(b, parity)) return true;
-  const uint64_t t0 = global_ns();
-  while (!mbar_try(b, parity)) {
-    if (global_ns() - t0 > kWaitLimitNs) {
-      atomicCAS(&g_tc_error, 0, code);
-      return false;
-    }
-  }
-  return true;
-}
-
-__device__ __forceinline__ float rn_tf32(float a) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(a));
-  return __uint_as_float(r);
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-      "[%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
-      : "memory");
-}
-
-// K-major, 128-byte swizzle shared-memory matrix descriptor (sm_100 layout):
-// start address >> 4 in [0,14), leading byte offset (unused here) in [16,30),
-// stride byte offset 1024 (8 rows x 128 B) >> 4 in [32,46), version 1 at [46,48),
-// layout type SWIZZLE_128B = 2 at [61,64).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= uint64_t((saddr & 0x3FFFF) >> 4);
-  d |= uint64_t(1) << 16;
-  d |= uint64_t(1024 >> 4) << 32;
-  d |= uint64_t(1) << 46;
-  d |= uint64_t(2) << 61;
-  return d;
-}
-
-// instruction descriptor of kind::tf32, fp32 accumulate, both operands K-major
-__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
-  return (1u << 4)                 // D format F32
-         | (2u << 7) | (2u << 10)  // A, B format TF32
-         | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc));
-}
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-template <int BN>
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+// bounded wait on the kernel's own pipeline; on expiry records `code` and returns false
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, uint64_t limit, int code) {
+  if (mbar_wait_for(b, parity, limit)) return true;
+  atomicCAS(&g_tc_error, 0, code);
+  return false;
 }
 
 template <int BN>
@@ -167,7 +76,8 @@ struct TcAcc {
 template <int BN, bool SPLIT>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const __grid_constant__ CUtensorMap tmBlo, int M, int N, int K, TcOut out, int accumulate) {
+              const __grid_constant__ CUtensorMap tmBlo, int M, int N, int K, TcOut out, int accumulate,
+              uint64_t limit) {
   using SM = TcSmem<BN>;
   constexpr int S = SM::kStages;
   constexpr uint32_t kCols = TcAcc<BN, SPLIT>::kCols;
@@ -197,14 +107,10 @@ __global__ void __launch_bounds__(192, 1)
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(kAlloc));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-  }
-  asm volatile("tcgen05.fence::before_thread_sync;");
+  if (warp == 1) tmem_alloc(tmem_slot, kAlloc);
+  fence_before_sync();
   __syncthreads();
-  asm volatile("tcgen05.fence::after_thread_sync;");
+  fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
   auto sA = [&](int s) { return base + s * SM::kStage; };
@@ -218,7 +124,7 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t bytes = SM::kA + (SPLIT ? 2 : 1) * SM::kB;
       for (int kt = 0; kt < nk; ++kt) {
         const int s = kt % S;
-        if (kt >= S && !mbar_wait(&empty[s], ((kt / S) + 1) & 1, 1)) {
+        if (kt >= S && !mbar_wait(&empty[s], ((kt / S) + 1) & 1, limit, 1)) {
           *abort_flag = 1;
           break;
         }
@@ -236,21 +142,21 @@ __global__ void __launch_bounds__(192, 1)
       for (int kt = 0; kt < nk; ++kt) {
         const int s = kt % S;
         const uint32_t par = (kt / S) & 1;
-        if (!mbar_wait(SPLIT ? &conv[s] : &full[s], par, 2) || *abort_flag) {
+        if (!mbar_wait(SPLIT ? &conv[s] : &full[s], par, limit, 2) || *abort_flag) {
           *abort_flag = 1;
           break;
         }
-        asm volatile("tcgen05.fence::after_thread_sync;");
+        fence_after_sync();
         const uint32_t a = smem_u32(sA(s)), al = smem_u32(sAlo(s)), b = smem_u32(sB(s)), bl = smem_u32(sBlo(s));
-#pragma unroll
         const uint32_t td = tmem + uint32_t((kt % NACC) * kCols);
+#pragma unroll
         for (int kk = 0; kk < kBK / 8; ++kk) {
           const uint32_t off = kk * 32;  // 8 TF32 = 32 bytes along K inside the swizzle atom
           const uint32_t acc = (kt >= NACC || kk > 0) ? 1u : 0u;
-          mma_tf32(td, sw128_desc(a + off), sw128_desc(b + off), idesc, acc);
+          mma_tf32(td, sw128_kmajor(a + off), sw128_kmajor(b + off), idesc, acc);
           if (SPLIT) {
-            mma_tf32(td, sw128_desc(a + off), sw128_desc(bl + off), idesc, 1u);
-            mma_tf32(td, sw128_desc(al + off), sw128_desc(b + off), idesc, 1u);
+            mma_tf32(td, sw128_kmajor(a + off), sw128_kmajor(bl + off), idesc, 1u);
+            mma_tf32(td, sw128_kmajor(al + off), sw128_kmajor(b + off), idesc, 1u);
           }
         }
         mma_commit(&empty[s]);
@@ -263,32 +169,20 @@ __global__ void __launch_bounds__(192, 1)
     if (SPLIT) {
       for (int kt = 0; kt < nk; ++kt) {
         const int s = kt % S;
-        if (!mbar_wait(&full[s], (kt / S) & 1, 3) || *abort_flag) {
+        if (!mbar_wait(&full[s], (kt / S) & 1, limit, 3) || *abort_flag) {
           *abort_flag = 1;
           break;
         }
         float4* a4 = reinterpret_cast<float4*>(sA(s));
         float4* l4 = reinterpret_cast<float4*>(sAlo(s));
 #pragma unroll 4
-        for (int i = t; i < kBM * kBK / 4; i += 128) {
-          float4 v = a4[i], h, l;
-          h.x = rn_tf32(v.x);
-          h.y = rn_tf32(v.y);
-          h.z = rn_tf32(v.z);
-          h.w = rn_tf32(v.w);
-          l.x = rn_tf32(v.x - h.x);
-          l.y = rn_tf32(v.y - h.y);
-          l.z = rn_tf32(v.z - h.z);
-          l.w = rn_tf32(v.w - h.w);
-          a4[i] = h;
-          l4[i] = l;
-        }
+        for (int i = t; i < kBM * kBK / 4; i += 128) split4(a4 + i, l4 + i);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive(&conv[s]);
       }
     }
-    const bool ok = mbar_wait(accf, 0, 4) && !*abort_flag;
-    asm volatile("tcgen05.fence::after_thread_sync;");
+    const bool ok = mbar_wait(accf, 0, limit, 4) && !*abort_flag;
+    fence_after_sync();
     if (ok) {
       const int q = warp & 3;  // TMEM lane quadrant this warp may access
       const int row = m0 + q * 32 + lane;
@@ -297,10 +191,10 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll 1
       for (int c = 0; c < BN; c += 16) {
         float v[16];
-        tmem_ld16<BN>(tmem + (uint32_t(q * 32) << 16) + uint32_t(c), v);
+        tmem_ld16(tmem + (uint32_t(q * 32) << 16) + uint32_t(c), v);
         for (int a = 1; a < nacc; ++a) {
           float w[16];
-          tmem_ld16<BN>(tmem + (uint32_t(q * 32) << 16) + uint32_t(a * kCols + c), w);
+          tmem_ld16(tmem + (uint32_t(q * 32) << 16) + uint32_t(a * kCols + c), w);
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] += w[i];
         }
@@ -337,13 +231,16 @@ __global__ void __launch_bounds__(192, 1)
   // drain: the producer waits (bounded) for the loads it issued so no copy is
   // in flight when the CTA exits, then TMEM is released
   if (warp == 0 && lane == 0 && *abort_flag) {
-    for (int kt = (issued > S ? issued - S : 0); kt < issued; ++kt) mbar_wait(&full[kt % S], (kt / S) & 1, 5);
+    for (int kt = (issued > S ? issued - S : 0); kt < issued; ++kt)
+      mbar_wait(&full[kt % S], (kt / S) & 1, kDrainLimitNs, 5);
   }
-  asm volatile("tcgen05.fence::before_thread_sync;");
+  // the MMA thread waits for its own MMAs before TMEM is released
+  if (warp == 1 && lane == 0) mbar_wait(accf, 0, kDrainLimitNs, 6);
+  fence_before_sync();
   __syncthreads();
   if (warp == 1) {
-    asm volatile("tcgen05.fence::after_thread_sync;");
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kAlloc));
+    fence_after_sync();
+    tmem_dealloc(tmem, kAlloc);
   }
 }
 
@@ -381,14 +278,14 @@ bool make_map(CUtensorMap* m, const float* p, int64_t rows, int64_t cols, int64_
 
 template <int BN, bool SPLIT>
 cudaError_t run(const float* A, int64_t lda, const float* B, const float* Blo, int64_t ldb, int M, int N, int K,
-                TcOut out, int accumulate, cudaStream_t st) {
+                TcOut out, int accumulate, uint64_t limit, cudaStream_t st) {
   CUtensorMap ta, tb, tbl;
   if (!make_map(&ta, A, M, K, lda, kBM) || !make_map(&tb, B, N, K, ldb, BN)) return cudaErrorInvalidValue;
   if (SPLIT && !make_map(&tbl, Blo, N, K, ldb, BN)) return cudaErrorInvalidValue;
   if (!SPLIT) tbl = tb;
   using SM = TcSmem<BN>;
   dim3 grid(unsigned((M + kBM - 1) / kBM), unsigned((N + BN - 1) / BN));
-  k_gemm_tc<BN, SPLIT><<<grid, 192, SM::kBytes, st>>>(ta, tb, tbl, M, N, K, out, accumulate);
+  k_gemm_tc<BN, SPLIT><<<grid, 192, SM::kBytes, st>>>(ta, tb, tbl, M, N, K, out, accumulate, limit);
   return cudaGetLastError();
 }
 
@@ -416,30 +313,29 @@ bool gemm_tc_supported(const float* A, int64_t lda, const float* B, int64_t ldb,
 }
 
 cudaError_t gemm_tc(const float* A, int64_t lda, const float* B, const float* Blo, int64_t ldb, int M, int N, int K,
-                    TcOut out, int accumulate, bool split, cudaStream_t st) {
+                    TcOut out, int accumulate, bool split, cudaStream_t st, uint64_t limit) {
   const int bn = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256));
   if (split) {
     switch (bn) {
-      case 32: return run<32, true>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
-      case 64: return run<64, true>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
-      case 128: return run<128, true>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
-      default: return run<256, true>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
+      case 32: return run<32, true>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, limit, st);
+      case 64: return run<64, true>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, limit, st);
+      case 128: return run<128, true>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, limit, st);
+      default: return run<256, true>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, limit, st);
     }
   }
   switch (bn) {
-    case 32: return run<32, false>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
-    case 64: return run<64, false>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
-    case 128: return run<128, false>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
-    default: return run<256, false>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, st);
+    case 32: return run<32, false>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, limit, st);
+    case 64: return run<64, false>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, limit, st);
+    case 128: return run<128, false>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, limit, st);
+    default: return run<256, false>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, limit, st);
   }
 }
 
-cudaError_t gemm_tc_read_error(int* code, cudaStream_t st) {
+cudaError_t gemm_tc_read_error(int* code) {
   int zero = 0;
-  cudaError_t e = cudaMemcpyFromSymbolAsync(code, g_tc_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st);
+  cudaError_t e = cudaMemcpyFromSymbol(code, g_tc_error, sizeof(int));
   if (e) return e;
-  if ((e = cudaStreamSynchronize(st))) return e;
-  return cudaMemcpyToSymbolAsync(g_tc_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+  return *code ? cudaMemcpyToSymbol(g_tc_error, &zero, sizeof(int)) : cudaSuccess;
 }
 
 // Theta^T split: hi[n][k] = rn_tf32(Theta[k][n]), lo = rn_tf32(Theta - hi)

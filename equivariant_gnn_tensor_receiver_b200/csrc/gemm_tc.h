@@ -19,8 +19,11 @@ cudaError_t gemm_tc_init();
 bool gemm_tc_supported(const float* A, int64_t lda, const float* B, int64_t ldb, int M, int N, int K);
 
 // C (+)= A[M][K] . B[N][K]^T.  split = 3xTF32 (B and Blo precomputed), else one TF32 pass.
+// limit: nanoseconds any wait on the kernel's own pipeline may take before the
+// kernel records an error (gemm_tc_read_error) and gives up.
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
 cudaError_t gemm_tc(const float* A, int64_t lda, const float* B, const float* Blo, int64_t ldb, int M, int N, int K,
-                    TcOut out, int accumulate, bool split, cudaStream_t st);
+                    TcOut out, int accumulate, bool split, cudaStream_t st, uint64_t limit = kDefaultWaitNs);
 
 // Theta block [K][N] -> hi = its transpose [N][K] (rounded to TF32 when lo != null), lo = remainder.
 cudaError_t split_transpose(const float* th, int K, int N, float* hi, float* lo, cudaStream_t st);
@@ -45,7 +48,8 @@ cudaError_t theta_x_pack_all(const float* th, const XPackList& l, float* hi, flo
 cudaError_t pack_rows(const float* g, int dim, int off, int mul, int n3, int64_t r0, int nc, float* out,
                       cudaStream_t st);
 
-// First error recorded by a bounded wait inside a tensor-core GEMM (0 = none); clears it. Synchronises st.
-cudaError_t gemm_tc_read_error(int* code, cudaStream_t st);
+// First error code recorded by an expired wait of a tensor-core GEMM since the
+// last read (0 = none); clears it.  The caller synchronises first.
+cudaError_t gemm_tc_read_error(int* code);
 
 }  // namespace tpc

@@ -18,6 +18,7 @@
 #include "plan.h"
 #include "wn_layout.h"
 #include "workspace.h"
+#include "dtheta_tc.h"
 
 using namespace tpc;
 
@@ -503,6 +504,14 @@ int tpc::ws_layout(const tpconv_plan& p, int op, int64_t N, int64_t E, WsLayout*
   L->off_lists = off;
   L->list_ints = work_list_ints(Nc);
   off = align256(off + size_t(kWorkLists) * L->list_ints * 4);
+  if (tc && op != TPCONV_OP_FORWARD && dtheta_tc_shape_ok(p.dp)) {
+    L->off_xt = off;
+    L->xt_bytes = align256(dtheta_tc_xt_floats(p.dp, Nc) * 4);
+    off += L->xt_bytes;
+    L->off_part = off;
+    L->part_bytes = align256(dtheta_tc_partial_floats(p.dp) * 4);
+    off += L->part_bytes;
+  }
   L->total = off;
   return TPCONV_OK;
 }

@@ -21,6 +21,7 @@
 #include "gemm_simt.cuh"
 #include "channelwise.h"
 #include "dtheta.h"
+#include "dtheta_tc.h"
 #include "gemm_tc.h"
 #include "graph.cuh"
 #include "launchers.h"
@@ -85,10 +86,16 @@ int ensure_device() {
   }
   if (dtheta_smem_init() != cudaSuccess) return TPCONV_ERR_CUDA;
   if (gemm_tc_init() != cudaSuccess) return TPCONV_ERR_CUDA;
+  if (dtheta_tc_init() != cudaSuccess) return TPCONV_ERR_CUDA;
   const unsigned long long now = current_context_id();  // the set-up above created the context if needed
   g_ready_ctx[dev] = now ? now : ~0ull;
   return TPCONV_OK;
 }
+
+// Limit of every wait of the tensor-core kernels on their own pipelines (set by
+// tpconv_set_wait_limit; read when a call is issued).
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+inline uint64_t wait_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 
 // 16-byte aligned (or null): the adjoint streams stage feature rows with 16-byte copies
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -252,7 +259,7 @@ cudaError_t node_mix_forward(const tpconv_plan* plan, int r0, int nc, const floa
       TcOut o{out + size_t(r0) * d.dim_out + d.out_off[i3], n3, d.dim_out, 1, n3};
       const bool split = plan->opt.gemm == TPCONV_GEMM_FP32;
       cudaError_t e = gemm_tc(Ab, Kb, thT_hi + toff, split ? thT_lo + toff : nullptr, Kb, int(M), cout, Kb, o,
-                              mode, split, si);
+                              mode, split, si, wait_ns());
       if (e) return e;
       continue;
     }
@@ -354,7 +361,7 @@ cudaError_t node_mix_adjoint(const tpconv_plan* plan, int r0, int nc, const floa
       TcOut o{Gb, 1, d.Kb[i3], 0, 1};
       const bool split = tc->N_lo != nullptr;
       if ((e = gemm_tc(gp, cout, tc->N_hi + toff, split ? tc->N_lo + toff : nullptr, cout, int(M), d.Kb[i3], cout,
-                       o, 0, split, si)))
+                       o, 0, split, si, wait_ns())))
         return e;
       continue;
     }
@@ -366,9 +373,30 @@ cudaError_t node_mix_adjoint(const tpconv_plan* plan, int r0, int nc, const floa
   return fj.join();
 }
 
+// dtheta += xa^T Ba (+ xb^T Bb) over the senders s0 : s0+nc: on the tensor
+// cores (deterministic split-K) where the workspace holds their regions, else
+// the FFMA kernel.
+cudaError_t theta_gradient(const tpconv_plan* plan, const WsLayout& L, void* ws, int s0, int nc, const float* xa,
+                           const float* Ba, const float* xb, const float* Bb, float* dtheta, cudaStream_t st) {
+  const DevPlan& d = plan->dp;
+  if (use_tc(plan) && L.xt_bytes > 0 && L.part_bytes > 0) {
+    char* w = static_cast<char*>(ws);
+    return dtheta_tc_accumulate(d, s0, nc, xa, Ba, xb, Bb, dtheta, reinterpret_cast<float*>(w + L.off_xt),
+                                reinterpret_cast<float*>(w + L.off_part), plan->opt.gemm == TPCONV_GEMM_FP32,
+                                wait_ns(), st);
+  }
+  return dtheta_accumulate(d, s0, nc, xa, Ba, xb, Bb, dtheta, st);
+}
+
+// kernel launches of theta_gradient: pack, GEMM and ordered reduce, or one FFMA kernel
+int64_t theta_gradient_launches(const tpconv_plan* plan, const WsLayout& L) {
+  return (use_tc(plan) && L.xt_bytes > 0 && L.part_bytes > 0) ? 3 : 1;
+}
+
 // dx[s0 : s0+nc] += B . Theta (per input block) and dtheta += x^T B (per path)
-cudaError_t node_mix_sender(const tpconv_plan* plan, int s0, int nc, const float* B, const float* x,
-                            const float* theta, const TcTheta* tc, float* dx, float* dtheta, cudaStream_t st) {
+cudaError_t node_mix_sender(const tpconv_plan* plan, const WsLayout& L, void* ws, int s0, int nc, const float* B,
+                            const float* x, const float* theta, const TcTheta* tc, float* dx, float* dtheta,
+                            cudaStream_t st) {
   const DevPlan& d = plan->dp;
   cudaError_t e;
   if (channelwise(plan)) {
@@ -390,7 +418,7 @@ cudaError_t node_mix_sender(const tpconv_plan* plan, int s0, int nc, const float
           TcOut o{dx + size_t(s0) * d.dim_in + d.in_off[i1], n1, d.dim_in, 1, n1};
           const bool split = tc->X_lo != nullptr;
           if ((e = gemm_tc(Bb, Kx, tc->X_hi + xo, split ? tc->X_lo + xo : nullptr, Kx, int(M), cin, Kx, o, 1, split,
-                           si)))
+                           si, wait_ns())))
             return e;
           continue;
         }
@@ -405,7 +433,7 @@ cudaError_t node_mix_sender(const tpconv_plan* plan, int s0, int nc, const float
       }
     }
   }
-  if (dtheta && (e = dtheta_accumulate(d, s0, nc, x, B, nullptr, nullptr, dtheta, st))) return e;
+  if (dtheta && (e = theta_gradient(plan, L, ws, s0, nc, x, B, nullptr, nullptr, dtheta, st))) return e;
   return fj.join();
 }
 
@@ -477,9 +505,40 @@ int finish(cudaError_t e) {
   return cudaGetLastError() == cudaSuccess ? TPCONV_OK : TPCONV_ERR_CUDA;
 }
 
+// Synchronises s, then reads and clears the error records of the tensor-core
+// kernels: TPCONV_ERR_TIMEOUT if a wait expired since the last read.
+int device_status(cudaStream_t s, int* status) {
+  *status = TPCONV_OK;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return TPCONV_ERR_CUDA;
+  int a = 0, b = 0;
+  if (gemm_tc_read_error(&a) != cudaSuccess || dtheta_tc_read_error(&b) != cudaSuccess) return TPCONV_ERR_CUDA;
+  if (a || b) *status = TPCONV_ERR_TIMEOUT;
+  return TPCONV_OK;
+}
+
+// end of a call: in validate mode the call waits for its kernels and reports an
+// expired device wait as TPCONV_ERR_TIMEOUT
+int finish_call(const tpconv_plan* plan, cudaStream_t s, cudaError_t e) {
+  const int st = finish(e);
+  if (st != TPCONV_OK || !plan->opt.validate) return st;
+  int dst = TPCONV_OK;
+  if (device_status(s, &dst) != TPCONV_OK) return TPCONV_ERR_CUDA;
+  return dst;
+}
+
 }  // namespace
 
 extern "C" {
+
+int tpconv_get_device_status(const tpconv_plan* plan, void* stream, int* status) {
+  if (!plan || !status) return TPCONV_ERR_INVALID_ARG;
+  return device_status(S(stream), status);
+}
+
+int tpconv_set_wait_limit(uint64_t ns) {
+  g_wait_ns.store(ns ? ns : kDefaultWaitNs, std::memory_order_relaxed);
+  return TPCONV_OK;
+}
 
 int tpconv_profile_enable(int on) {
   prof().on = on != 0;
@@ -600,7 +659,7 @@ int tpconv_forward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t*
       note(TPCONV_PHASE_FWD_NODE, d.n_out);
     }
   }
-  return finish(cudaSuccess);
+  return finish_call(plan, s, cudaSuccess);
 }
 
 int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t* rowptr, const int32_t* col,
@@ -672,13 +731,15 @@ int tpconv_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t
       }
       {
         PhaseScope ps(TPCONV_PHASE_BWD_NODE_X, s);
-        if (node_mix_sender(plan, int(s0), nc, S_, x, theta, tcp, dx, dtheta, s)) return TPCONV_ERR_CUDA;
+        if (node_mix_sender(plan, L, workspace, int(s0), nc, S_, x, theta, tcp, dx, dtheta, s))
+          return TPCONV_ERR_CUDA;
         const int64_t nx = channelwise(plan) ? cw_launches_in(d) : d.n_in;
-        note(TPCONV_PHASE_BWD_NODE_X, int64_t(dx ? nx : 0) + int64_t(dtheta ? (channelwise(plan) ? nx : 1) : 0));
+        note(TPCONV_PHASE_BWD_NODE_X, int64_t(dx ? nx : 0) +
+                                          int64_t(dtheta ? (channelwise(plan) ? nx : theta_gradient_launches(plan, L)) : 0));
       }
     }
   }
-  return finish(cudaSuccess);
+  return finish_call(plan, s, cudaSuccess);
 }
 
 int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const int32_t* rowptr,
@@ -798,21 +859,28 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
       PhaseScope ps(TPCONV_PHASE_DBL_NODE_X, s);
       float* dx1 = has_v ? d_x : nullptr;
       float* dt1 = has_v ? d_theta : nullptr;
-      if (dx1 && node_mix_sender(plan, int(s0), nc, B1, x, theta, tc0p, dx1, nullptr, s)) return TPCONV_ERR_CUDA;
+      if (dx1 && node_mix_sender(plan, L, workspace, int(s0), nc, B1, x, theta, tc0p, dx1, nullptr, s))
+        return TPCONV_ERR_CUDA;
       float* dx0 = has_t ? d_x : nullptr;
       float* dt0 = has_x1 ? d_theta : nullptr;
-      if (dx0 && node_mix_sender(plan, int(s0), nc, B0, gg_x, gg_theta, tc1p, dx0, nullptr, s)) return TPCONV_ERR_CUDA;
-      // d_theta = x^T B1 + gg_x^T B0 in one pass
-      if ((dt1 || dt0) &&
-          (channelwise(plan) ? cw_dtheta : dtheta_accumulate)(d, int(s0), nc, dt1 ? x : nullptr, dt1 ? B1 : nullptr,
-                                                              dt0 ? gg_x : nullptr, dt0 ? B0 : nullptr, d_theta, s))
+      if (dx0 && node_mix_sender(plan, L, workspace, int(s0), nc, B0, gg_x, gg_theta, tc1p, dx0, nullptr, s))
         return TPCONV_ERR_CUDA;
+      // d_theta = x^T B1 + gg_x^T B0 in one pass
+      if (dt1 || dt0) {
+        const float *xa = dt1 ? x : nullptr, *Ba = dt1 ? B1 : nullptr;
+        const float *xb = dt0 ? gg_x : nullptr, *Bb = dt0 ? B0 : nullptr;
+        const cudaError_t e = channelwise(plan) ? cw_dtheta(d, int(s0), nc, xa, Ba, xb, Bb, d_theta, s)
+                                                : theta_gradient(plan, L, workspace, int(s0), nc, xa, Ba, xb, Bb,
+                                                                 d_theta, s);
+        if (e) return TPCONV_ERR_CUDA;
+      }
       const int64_t nx = channelwise(plan) ? cw_launches_in(d) : d.n_in;
       note(TPCONV_PHASE_DBL_NODE_X,
-           int64_t(dx1 ? nx : 0) + int64_t(dx0 ? nx : 0) + ((dt1 || dt0) ? (channelwise(plan) ? nx : 1) : 0));
+           int64_t(dx1 ? nx : 0) + int64_t(dx0 ? nx : 0) +
+               ((dt1 || dt0) ? (channelwise(plan) ? nx : theta_gradient_launches(plan, L)) : 0));
     }
   }
-  return finish(cudaSuccess);
+  return finish_call(plan, s, cudaSuccess);
 }
 
 }  // extern "C"

@@ -16,6 +16,8 @@ struct WsLayout {
   size_t off_pack, pack_bytes;     // one packed feature block of a chunk (tensor-core A operand)
   size_t off_cursor, off_scan, off_tmp;  // graph transpose scratch
   size_t off_lists, list_ints;     // work lists of the edge streams: kWorkLists x list_ints ints
+  size_t off_xt, xt_bytes;         // tensor-core Theta gradient: packed x of a chunk (2 pairs x {hi, lo})
+  size_t off_part, part_bytes;     // tensor-core Theta gradient: partial tiles of one call
 };
 
 // Work lists of one chunk (receiver pieces, receiver batches, sender pieces),

@@ -68,7 +68,7 @@ extern "C" {
 #define TPCONV_ERR_WORKSPACE_TOO_SMALL 4
 #define TPCONV_ERR_CUDA 5               /* a CUDA runtime call failed           */
 #define TPCONV_ERR_GRAPH_INVALID 6      /* validate mode: bad CSR / indices     */
-#define TPCONV_ERR_TIMEOUT 7            /* reserved: bounded device wait expired */
+#define TPCONV_ERR_TIMEOUT 7            /* a bounded device wait expired        */
 #define TPCONV_ERR_INTERNAL 8           /* self-check failed (e.g. CG table)    */
 
 /* radial basis kinds */
@@ -246,6 +246,30 @@ int tpconv_double_backward(const tpconv_plan* plan, int64_t N, int64_t E, const 
                            const float* gg_vec, const float* gg_theta, float* d_g, float* d_x,
                            float* d_vec, float* d_theta, void* workspace, size_t workspace_bytes,
                            void* stream);
+
+/*
+ * Device-side wait status (host; synchronises the stream).  The tensor-core
+ * kernels (Theta contractions and Theta gradient) wait only on their own
+ * pipelines (TMA copies into shared memory, tensor-core MMAs), and every such
+ * wait is bounded by a time limit.  When one expires the kernel records it,
+ * stops issuing work, waits (bounded) for the copies and MMAs it has already
+ * issued, frees its tensor memory and returns; its output is then not valid.
+ * No kernel of the library waits on another CTA, kernel or GPU.
+ *   *status = TPCONV_ERR_TIMEOUT if a wait expired since the previous query
+ *   (the record is cleared), else TPCONV_OK.  Returns TPCONV_ERR_CUDA if the
+ *   stream or the query itself fails.
+ * With tpconv_options.validate set, every forward / backward / double backward
+ * ends with this query and returns its status.  Not defined in the pages: an
+ * interface addition for failure detection.
+ */
+int tpconv_get_device_status(const tpconv_plan* plan, void* stream, int* status);
+
+/*
+ * Limit of those device waits, in nanoseconds, for calls issued from now on
+ * (process-wide; 0 restores the default of 2 s).  Tests use a tiny limit to
+ * make the waits run out on purpose and check the error path.
+ */
+int tpconv_set_wait_limit(uint64_t ns);
 
 /*
  * Diagnostics (host).  Every kernel launch of the library is counted per phase.

@@ -109,10 +109,13 @@ def test_workspace_independent_of_edges_and_capped(T):
     cap = 64 << 20
     capped = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], workspace_cap=cap)
     theta_ops = 12 * 4 * capped.theta_numel  # tensor-core Theta operands: independent of N and E
+    # the tensor-core Theta gradient adds x of one chunk (4 x dim_in floats per
+    # node, against the node state's 22016) and a fixed buffer of partial tiles
+    partials = 2 * 160 * 64 * 128 * 4
     for op in (0, 1, 2):
         big = T.tpconv_workspace_size(capped, op, 1_222_309, 64_000_000)
         assert big == T.tpconv_workspace_size(capped, op, 500_000, 1_000)
-        assert big <= cap + theta_ops + (4 << 20)
+        assert big <= cap * (1 + 4 * 576 / 22016) + theta_ops + partials + (4 << 20)
 
 
 def test_bf16_mixing_is_reported_unsupported(T):
@@ -137,8 +140,13 @@ def test_theta_region_sized_per_operation(T, gemm, per_op):
 
     plan, a = size(1)           # one node per chunk: the Theta region dominates
     tn = (plan.theta_numel + 63) // 64 * 64 * 4
-    for got, k in zip(a, per_op):
-        assert k * tn <= got <= k * tn + (1 << 20), (got, k * tn)
+    # backward and double backward on tensor cores also hold the Theta
+    # gradient's partial tiles: one 128 x 128 tile per row tile of both operand
+    # pairs (23 paths x 8 row tiles x 2), at least two waves of 160
+    part = max(2 * 160, 2 * 23 * 8) * 128 * 128 * 4 if gemm != "simt" else 0
+    for op, (got, k) in enumerate(zip(a, per_op)):
+        extra = part if op > 0 else 0
+        assert k * tn + extra <= got <= k * tn + extra + (1 << 20), (op, got, k * tn + extra)
     _, b = size(0)
     state = 4 * 8192 * 101_376  # A floats per node of the wide layer
     assert b[0] >= state + per_op[0] * tn
