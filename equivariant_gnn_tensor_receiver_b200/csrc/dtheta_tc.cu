@@ -14,10 +14,10 @@
 //
 //   A operand = the sender-side state B, read in place.  Along a row of B the
 //               (k, w) columns are contiguous, so A is "MN-major": TMA loads
-//               32 (M) x 32 (K) boxes with the 128-byte swizzle, four per
-//               128-row tile, and the MMA reads them through MN-major
-//               descriptors (atoms of 8 K-rows x 128 bytes; 4096 bytes between
-//               atoms along M, 1024 along K).
+//               32 (M) x 32 (K) boxes, four per 128-row tile, in the layout
+//               the tensor core takes for MN-major TF32 operands (128-byte
+//               swizzle with 32-byte atomicity: atoms of 4 K-rows x 128 bytes;
+//               4096 bytes between atoms along M, 512 along K).
 //   B operand = Xt[u][K], x of the chunk transposed per input block (K-major),
 //               packed by k_pack_xt (already split into TF32 hi / lo).
 //
@@ -78,7 +78,7 @@ struct DtGroup {
 };
 
 struct __align__(64) DtParams {
-  CUtensorMap a[kMaxMaps];   // B state [K][Kx] of (pair, i1), box 32 x 32, SW128
+  CUtensorMap a[kMaxMaps];   // B state [K][Kx] of (pair, i1), box 32 x 32, 128-byte swizzle, 32-byte atoms
   CUtensorMap bh[kMaxMaps];  // Xt hi [c_in][K], box 32 x BN, SW128
   CUtensorMap bl[kMaxMaps];  // Xt lo (3xTF32 only)
   DtGroup g[kMaxGroups];
@@ -96,11 +96,15 @@ struct DtSmem {
   static constexpr int kBytes = kStages * kStage + 1024 + 256;
 };
 
+// TMEM accumulators; 3xTF32 with column tiles of at most 128 runs the round
+// schedule of tc_common.cuh (accumulation chains of 4 K steps, rounds added
+// into fp32 registers), which keeps fp32 accuracy for the long K of this GEMM.
 template <int BN, bool SPLIT>
 struct DtAcc {
   static constexpr int kCols = BN < 32 ? 32 : BN;
   static constexpr int N = SPLIT ? (512 / kCols > 8 ? 8 : 512 / kCols) : 1;
   static constexpr uint32_t kAlloc = kCols * N;
+  static constexpr bool kDrain = SPLIT && BN <= 128;
 };
 
 // record the first error of the launch and report expiry
@@ -117,6 +121,8 @@ __global__ void __launch_bounds__(192, 1) k_dtheta_tc(const __grid_constant__ Dt
   constexpr uint32_t kCols = DtAcc<BN, SPLIT>::kCols;
   constexpr int NACC = DtAcc<BN, SPLIT>::N;
   constexpr uint32_t kAlloc = DtAcc<BN, SPLIT>::kAlloc;
+  constexpr bool DRAIN = DtAcc<BN, SPLIT>::kDrain;
+  using RS = Rounds<NACC>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -124,7 +130,9 @@ __global__ void __launch_bounds__(192, 1) k_dtheta_tc(const __grid_constant__ Dt
   uint64_t* conv = full + S;
   uint64_t* empty = conv + S;
   uint64_t* accf = empty + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  uint64_t* bfull = accf + 1;   // [2] a round of the bank is complete
+  uint64_t* bfree = bfull + 2;  // [2] the bank has been added into registers
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bfree + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -148,6 +156,10 @@ __global__ void __launch_bounds__(192, 1) k_dtheta_tc(const __grid_constant__ Dt
       mbar_init(&empty[s], 1);
     }
     mbar_init(accf, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bfull[b], 1);
+      mbar_init(&bfree[b], 128);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -190,35 +202,62 @@ __global__ void __launch_bounds__(192, 1) k_dtheta_tc(const __grid_constant__ Dt
       constexpr uint32_t idesc = idesc_tf32(kBM, BN, /*a_mn=*/true, /*b_mn=*/false);
       for (int kt = 0; kt < nk; ++kt) {
         const int s = kt % S;
+        const int r = DRAIN ? kt / RS::D : 0, j = DRAIN ? kt - r * RS::D : kt, bank = r & 1;
+        if (DRAIN && j == 0 && r >= 2 && !waitp(&bfree[bank], ((r >> 1) - 1) & 1, limit, 7)) {
+          *abort_flag = 1;
+          break;
+        }
         if (!waitp(SPLIT ? &conv[s] : &full[s], (kt / S) & 1, limit, 2) || *abort_flag) {
           *abort_flag = 1;
           break;
         }
         fence_after_sync();
         const uint32_t a = smem_u32(sA(s)), al = smem_u32(sAlo(s)), b = smem_u32(sB(s)), bl = smem_u32(sBlo(s));
-        const uint32_t td = tmem + uint32_t((kt % NACC) * kCols);
+        const int ai = DRAIN ? bank * RS::NPB + j % RS::NPB : kt % NACC;
+        const int fresh = DRAIN ? RS::NPB : NACC;  // the first steps of a round (of the CTA) overwrite
+        const uint32_t td = tmem + uint32_t(ai * kCols);
 #pragma unroll
         for (int kk = 0; kk < kBK / 8; ++kk) {
-          // A: 8 K-rows per MMA = one 1024-byte atom row; B: 8 TF32 = 32 bytes along K
-          const uint64_t da = sw128_desc(a + kk * 1024, 4096, 1024);
+          // A: 8 K-rows per MMA = two 512-byte atoms along K; B: 8 TF32 = 32 bytes along K
+          const uint64_t da = sw128b32_mn_desc(a + kk * 1024, 4096, 512);
           const uint64_t db = sw128_kmajor(b + kk * 32);
-          const uint32_t acc = (kt >= NACC || kk > 0) ? 1u : 0u;
+          const uint32_t acc = (j >= fresh || kk > 0) ? 1u : 0u;
           mma_tf32(td, da, db, idesc, acc);
           if (SPLIT) {
             mma_tf32(td, da, sw128_kmajor(bl + kk * 32), idesc, 1u);
-            mma_tf32(td, sw128_desc(al + kk * 1024, 4096, 1024), db, idesc, 1u);
+            mma_tf32(td, sw128b32_mn_desc(al + kk * 1024, 4096, 512), db, idesc, 1u);
           }
         }
         mma_commit(&empty[s]);
+        if (DRAIN && (j == RS::D - 1 || kt == nk - 1)) mma_commit(&bfull[bank]);
       }
       mma_commit(accf);  // fires once every MMA issued above has completed
     }
   } else {
+    // warps 2..5: split A (3xTF32), add finished rounds into registers, store
+    // the partial tile; exit decisions are warp-uniform (TMEM loads are
+    // warp-collective)
     const int t = threadIdx.x - 64;  // 0..127
+    const int q = warp & 3;          // TMEM lane quadrant of this warp
+    const uint32_t tlane = tmem + (uint32_t(q * 32) << 16);
+    constexpr int NR = DRAIN ? BN : 16;
+    float racc[NR];
+#pragma unroll
+    for (int i = 0; i < NR; ++i) racc[i] = 0.f;
+    int drained = 0;
+    auto drain = [&](int rr) -> bool {
+      if (!__all_sync(0xffffffffu, waitp(&bfull[rr & 1], (rr >> 1) & 1, limit, 8))) return false;
+      fence_after_sync();
+      tmem_drain<NR, RS::NPB>(tlane, rr & 1, min(RS::NPB, RS::steps(rr, nk)), kCols, racc);
+      fence_before_sync();
+      mbar_arrive(&bfree[rr & 1]);
+      ++drained;
+      return true;
+    };
     if (SPLIT) {
       for (int kt = 0; kt < nk; ++kt) {
         const int s = kt % S;
-        if (!waitp(&full[s], (kt / S) & 1, limit, 3) || *abort_flag) {
+        if (!__all_sync(0xffffffffu, waitp(&full[s], (kt / S) & 1, limit, 3) && !*abort_flag)) {
           *abort_flag = 1;
           break;
         }
@@ -228,22 +267,35 @@ __global__ void __launch_bounds__(192, 1) k_dtheta_tc(const __grid_constant__ Dt
         for (int i = t; i < kBM * kBK / 4; i += 128) split4(a4 + i, l4 + i);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive(&conv[s]);
+        if constexpr (DRAIN) {
+          const int rr = RS::drain_after(kt);
+          if (rr >= 0 && !drain(rr)) {
+            *abort_flag = 1;
+            break;
+          }
+        }
       }
     }
-    const bool ok = waitp(accf, 0, limit, 4) && !*abort_flag;
+    bool ok = __all_sync(0xffffffffu, waitp(accf, 0, limit, 4) && !*abort_flag);
     fence_after_sync();
-    const int q = warp & 3;  // TMEM lane quadrant of this warp
+    if constexpr (DRAIN) {
+      const int nrounds = (nk + RS::D - 1) / RS::D;
+      while (ok && drained < nrounds) ok = drain(drained);
+    }
     const int row = q * 32 + lane;
     float* dst = P.partial + size_t(blockIdx.x) * BN * kBM + row;
     const int nacc = nk < NACC ? nk : NACC;
-#pragma unroll 1
+#pragma unroll
     for (int c = 0; c < BN; c += 16) {
       float v[16];
-      if (ok && nk > 0) {
-        tmem_ld16(tmem + (uint32_t(q * 32) << 16) + uint32_t(c), v);
+      if (ok && nk > 0 && DRAIN) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = racc[(c + i) % NR];
+      } else if (ok && nk > 0) {
+        tmem_ld16(tlane + uint32_t(c), v);
         for (int a = 1; a < nacc; ++a) {
           float w[16];
-          tmem_ld16(tmem + (uint32_t(q * 32) << 16) + uint32_t(a * kCols + c), w);
+          tmem_ld16(tlane + uint32_t(a * kCols + c), w);
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] += w[i];
         }
@@ -359,8 +411,9 @@ EncodeFn encoder() {
   return fn;
 }
 
-// fp32 [rows][cols] with row pitch ld floats; box box_cols x box_rows, 128-byte swizzle
-bool make_map(CUtensorMap* m, const float* p, int64_t rows, int64_t cols, int64_t ld, int box_cols, int box_rows) {
+// fp32 [rows][cols] with row pitch ld floats; box box_cols x box_rows
+bool make_map(CUtensorMap* m, const float* p, int64_t rows, int64_t cols, int64_t ld, int box_cols, int box_rows,
+              CUtensorMapSwizzle swz) {
   EncodeFn enc = encoder();
   if (!enc) return false;
   if ((reinterpret_cast<uintptr_t>(p) & 15) || ((ld * 4) & 15) || rows <= 0 || cols <= 0) return false;
@@ -369,7 +422,7 @@ bool make_map(CUtensorMap* m, const float* p, int64_t rows, int64_t cols, int64_
   cuuint32_t box[2] = {cuuint32_t(box_cols), cuuint32_t(box_rows)};
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(p), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -519,9 +572,9 @@ cudaError_t dtheta_tc_accumulate(const DevPlan& d, int s0, int nc, const float* 
       const float* xh = xp.hi[pr] + xp.b[i1].off;
       const float* xl = split ? xp.lo[pr] + xp.b[i1].off : xh;
       const int64_t K = int64_t(nc) * n1, kp = kpad_of(nc, n1);
-      if (!make_map(&dp.a[nmap], Bst, K, d.Kx[i1], d.Kx[i1], 32, 32) ||
-          !make_map(&dp.bh[nmap], xh, d.in_mul[i1], K, kp, 32, BN) ||
-          !make_map(&dp.bl[nmap], xl, d.in_mul[i1], K, kp, 32, BN))
+      if (!make_map(&dp.a[nmap], Bst, K, d.Kx[i1], d.Kx[i1], 32, 32, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) ||
+          !make_map(&dp.bh[nmap], xh, d.in_mul[i1], K, kp, 32, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !make_map(&dp.bl[nmap], xl, d.in_mul[i1], K, kp, 32, BN, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
       mapped[pr][i1] = nmap++;
     }

@@ -60,17 +60,19 @@ struct TcSmem {
   static constexpr int kB = BN * kBK * 4;    // BN x 128 B
   static constexpr int kStage = 2 * kA + 2 * kB;
   static constexpr int kStages = (200 * 1024) / kStage >= 4 ? 4 : ((200 * 1024) / kStage >= 3 ? 3 : 2);
-  static constexpr int kBytes = kStages * kStage + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kBytes = kStages * kStage + 1024 /*align*/ + 256 /*barriers: 3 x stages + 5, slot, flag*/;
 };
 
-// Accumulators in TMEM: the 3xTF32 mode spreads consecutive K steps over NACC
-// accumulators (summed in fp32 by the epilogue), so each one sees 1/NACC of
-// the accumulation steps; this bounds the error the accumulation itself adds.
+// Accumulators in TMEM.  The 3xTF32 mode uses NACC of them in the round
+// schedule of tc_common.cuh (chains of 4 K steps, rounds added into fp32
+// registers), for column tiles of at most 128; with 256 columns (only used for
+// short K) the K steps alternate over two accumulators summed at the end.
 template <int BN, bool SPLIT>
 struct TcAcc {
   static constexpr int kCols = BN < 32 ? 32 : BN;
   static constexpr int N = SPLIT ? (512 / kCols > 8 ? 8 : 512 / kCols) : 1;
   static constexpr uint32_t kAlloc = kCols * N;  // power of two, <= 512
+  static constexpr bool kDrain = SPLIT && BN <= 128;
 };
 
 template <int BN, bool SPLIT>
@@ -83,13 +85,17 @@ __global__ void __launch_bounds__(192, 1)
   constexpr uint32_t kCols = TcAcc<BN, SPLIT>::kCols;
   constexpr int NACC = TcAcc<BN, SPLIT>::N;
   constexpr uint32_t kAlloc = TcAcc<BN, SPLIT>::kAlloc;
+  constexpr bool DRAIN = TcAcc<BN, SPLIT>::kDrain;
+  using RS = Rounds<NACC>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(base + S * SM::kStage);
   uint64_t* conv = full + S;
   uint64_t* empty = conv + S;
   uint64_t* accf = empty + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  uint64_t* bfull = accf + 1;  // [2] a round of the bank is complete (round schedule)
+  uint64_t* bfree = bfull + 2; // [2] the bank has been added into registers
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bfree + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -104,6 +110,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(accf, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bfull[b], 1);
+      mbar_init(&bfree[b], 128);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -142,17 +152,25 @@ __global__ void __launch_bounds__(192, 1)
       for (int kt = 0; kt < nk; ++kt) {
         const int s = kt % S;
         const uint32_t par = (kt / S) & 1;
+        // round schedule: round r = kt / D writes bank r & 1, free again once round r - 2 was drained
+        const int r = DRAIN ? kt / RS::D : 0, j = DRAIN ? kt - r * RS::D : kt, bank = r & 1;
+        if (DRAIN && j == 0 && r >= 2 && !mbar_wait(&bfree[bank], ((r >> 1) - 1) & 1, limit, 7)) {
+          *abort_flag = 1;
+          break;
+        }
         if (!mbar_wait(SPLIT ? &conv[s] : &full[s], par, limit, 2) || *abort_flag) {
           *abort_flag = 1;
           break;
         }
         fence_after_sync();
         const uint32_t a = smem_u32(sA(s)), al = smem_u32(sAlo(s)), b = smem_u32(sB(s)), bl = smem_u32(sBlo(s));
-        const uint32_t td = tmem + uint32_t((kt % NACC) * kCols);
+        const int ai = DRAIN ? bank * RS::NPB + j % RS::NPB : kt % NACC;
+        const int fresh = DRAIN ? RS::NPB : NACC;  // the first `fresh` steps of a round (of the call) overwrite
+        const uint32_t td = tmem + uint32_t(ai * kCols);
 #pragma unroll
         for (int kk = 0; kk < kBK / 8; ++kk) {
           const uint32_t off = kk * 32;  // 8 TF32 = 32 bytes along K inside the swizzle atom
-          const uint32_t acc = (kt >= NACC || kk > 0) ? 1u : 0u;
+          const uint32_t acc = (j >= fresh || kk > 0) ? 1u : 0u;
           mma_tf32(td, sw128_kmajor(a + off), sw128_kmajor(b + off), idesc, acc);
           if (SPLIT) {
             mma_tf32(td, sw128_kmajor(a + off), sw128_kmajor(bl + off), idesc, 1u);
@@ -160,16 +178,36 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
         mma_commit(&empty[s]);
+        if (DRAIN && (j == RS::D - 1 || kt == nk - 1)) mma_commit(&bfull[bank]);
       }
       mma_commit(accf);
     }
   } else {
-    // warps 2..5: split A in shared memory (3xTF32), then the epilogue
+    // warps 2..5: split A in shared memory (3xTF32), add finished rounds of
+    // accumulators into registers, then the epilogue
     const int t = threadIdx.x - 64;  // 0..127
+    const int q = warp & 3;          // TMEM lane quadrant this warp may access
+    const uint32_t tlane = tmem + (uint32_t(q * 32) << 16);
+    constexpr int NR = DRAIN ? BN : 16;  // register accumulators (unused without the round schedule)
+    float racc[NR];
+#pragma unroll
+    for (int i = 0; i < NR; ++i) racc[i] = 0.f;
+    int drained = 0;  // rounds added into racc
+    // every exit decision of these warps is made warp-uniform (__all_sync): the
+    // TMEM loads below are warp-collective
+    auto drain = [&](int rr) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bfull[rr & 1], (rr >> 1) & 1, limit, 8))) return false;
+      fence_after_sync();
+      tmem_drain<NR, RS::NPB>(tlane, rr & 1, min(RS::NPB, RS::steps(rr, nk)), kCols, racc);
+      fence_before_sync();
+      mbar_arrive(&bfree[rr & 1]);
+      ++drained;
+      return true;
+    };
     if (SPLIT) {
       for (int kt = 0; kt < nk; ++kt) {
         const int s = kt % S;
-        if (!mbar_wait(&full[s], (kt / S) & 1, limit, 3) || *abort_flag) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (kt / S) & 1, limit, 3) && !*abort_flag)) {
           *abort_flag = 1;
           break;
         }
@@ -179,24 +217,39 @@ __global__ void __launch_bounds__(192, 1)
         for (int i = t; i < kBM * kBK / 4; i += 128) split4(a4 + i, l4 + i);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive(&conv[s]);
+        if constexpr (DRAIN) {
+          const int rr = RS::drain_after(kt);
+          if (rr >= 0 && !drain(rr)) {
+            *abort_flag = 1;
+            break;
+          }
+        }
       }
     }
-    const bool ok = mbar_wait(accf, 0, limit, 4) && !*abort_flag;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(accf, 0, limit, 4) && !*abort_flag);
     fence_after_sync();
+    if constexpr (DRAIN) {
+      const int nrounds = (nk + RS::D - 1) / RS::D;
+      while (ok && drained < nrounds) ok = drain(drained);
+    }
     if (ok) {
-      const int q = warp & 3;  // TMEM lane quadrant this warp may access
       const int row = m0 + q * 32 + lane;
       const int64_t rbase = (row / out.rdiv) * out.r_hi + (row % out.rdiv) * out.r_lo;
       const int nacc = nk < NACC ? nk : NACC;  // accumulators that received a K step
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < BN; c += 16) {
         float v[16];
-        tmem_ld16(tmem + (uint32_t(q * 32) << 16) + uint32_t(c), v);
-        for (int a = 1; a < nacc; ++a) {
-          float w[16];
-          tmem_ld16(tmem + (uint32_t(q * 32) << 16) + uint32_t(a * kCols + c), w);
+        if constexpr (DRAIN) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] += w[i];
+          for (int i = 0; i < 16; ++i) v[i] = racc[(c + i) % NR];
+        } else {
+          tmem_ld16(tlane + uint32_t(c), v);
+          for (int a = 1; a < nacc; ++a) {
+            float w[16];
+            tmem_ld16(tlane + uint32_t(a * kCols + c), w);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] += w[i];
+          }
         }
         if (row < M) {
           float* dst0 = out.p + rbase + int64_t(n0 + c) * out.c_hi;
@@ -314,7 +367,9 @@ bool gemm_tc_supported(const float* A, int64_t lda, const float* B, int64_t ldb,
 
 cudaError_t gemm_tc(const float* A, int64_t lda, const float* B, const float* Blo, int64_t ldb, int M, int N, int K,
                     TcOut out, int accumulate, bool split, cudaStream_t st, uint64_t limit) {
-  const int bn = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256));
+  // 3xTF32 with long K uses column tiles of at most 128, whose accumulators are
+  // drained into registers in rounds (bounded TMEM accumulation chains)
+  const int bn = N <= 32 ? 32 : (N <= 64 ? 64 : ((N <= 128 || (split && K > 256)) ? 128 : 256));
   if (split) {
     switch (bn) {
       case 32: return run<32, true>(A, lda, B, Blo, ldb, M, N, K, out, accumulate, limit, st);

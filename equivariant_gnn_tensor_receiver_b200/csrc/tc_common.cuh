@@ -76,9 +76,7 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
 // [32,46), version 1 at [46,48), layout SWIZZLE_128B = 2 at [61,64).
 //   K-major operand : 8-row x 128-byte atoms stacked along the rows (SBO = 1024);
 //                     the leading offset is unused.
-//   MN-major operand: atoms of 8 K-rows x 128 bytes (32 fp32 along M or N);
-//                     LBO = bytes between atoms along M / N, SBO = bytes between
-//                     atoms along K.
+//   (MN-major TF32 operands need the 32-byte-atom variant below.)
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
   uint64_t d = 0;
   d |= uint64_t((saddr & 0x3FFFF) >> 4);
@@ -89,6 +87,22 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
   return d;
 }
 __device__ __forceinline__ uint64_t sw128_kmajor(uint32_t saddr) { return sw128_desc(saddr, 16, 1024); }
+
+// MN-major TF32 operands take the one layout the tensor core accepts for them:
+// the 128-byte swizzle with 32-byte atomicity (layout type 1 at [61,64); TMA's
+// CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B writes it).  Atoms of 4 K-rows x 128 bytes
+// (32 fp32 along M / N), the 32-byte pieces of a row permuted by the row index
+// mod 4.  LBO = bytes between atoms along M / N, SBO = bytes between 4-row
+// groups along K.
+__device__ __forceinline__ uint64_t sw128b32_mn_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr & 0x3FFFF) >> 4);
+  d |= uint64_t((lbo_bytes >> 4) & 0x3FFF) << 16;
+  d |= uint64_t((sbo_bytes >> 4) & 0x3FFF) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(1) << 61;
+  return d;
+}
 
 // Instruction descriptor of kind::tf32 with fp32 accumulation: D format F32 at
 // [4,6), A and B format TF32 at [7,10) and [10,13), A / B major-ness at bits 15
@@ -148,6 +162,45 @@ __device__ __forceinline__ void split4(float4* a, float4* lo) {
   l.w = rn_tf32(v.w - h.w);
   *a = h;
   *lo = l;
+}
+
+// ---- accumulation schedule of the 3xTF32 kernels ------------------------------
+// The tensor core accumulates in fp32 inside TMEM; its rounding error grows with
+// the length of an accumulation chain, i.e. with K.  The NACC accumulators form
+// two banks of NPB.  K steps run in rounds of D = 4 NPB steps; round r writes
+// bank r & 1, each accumulator starting afresh and taking every NPB-th step, so
+// no chain is longer than 4 K steps (48 MMAs of K = 8).  The epilogue warps add
+// a finished round's bank into fp32 registers (round to nearest) halfway through
+// the next round and release the bank for round r + 2; a round's last MMA
+// commits to bank_full, the drain arrives on bank_free.
+template <int NACC>
+struct Rounds {
+  static constexpr int NPB = NACC / 2;  // accumulators per bank
+  static constexpr int D = 4 * NPB;     // K steps per round
+  __device__ static int steps(int r, int nk) { return min(D, nk - r * D); }
+  // the converter / epilogue warps drain round r right after handling K step kt, or -1
+  __device__ static int drain_after(int kt) {
+    const int t = kt + 1 - D / 2;
+    return (t >= D && t % D == 0) ? t / D - 1 : -1;
+  }
+};
+
+// add the accumulators of one bank that a round wrote (n_used <= NPB, warp-uniform)
+// into racc; tlane = TMEM address of this warp's lane quadrant, column 0
+template <int BN, int NPB>
+__device__ __forceinline__ void tmem_drain(uint32_t tlane, int bank, int n_used, uint32_t cols, float (&racc)[BN]) {
+#pragma unroll
+  for (int c = 0; c < BN; c += 16) {
+#pragma unroll
+    for (int a = 0; a < NPB; ++a) {
+      if (a < n_used) {
+        float w[16];
+        tmem_ld16(tlane + uint32_t((bank * NPB + a) * cols + c), w);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) racc[c + i] += w[i];
+      }
+    }
+  }
 }
 
 }  // namespace tc
