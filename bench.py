@@ -77,6 +77,10 @@ def parse():
                          "fwd, fwd+bwd and double-bwd edges/s, peak memory, roofline of the dominant kernel")
     ap.add_argument("--suite-configs", default="tiny,mace,sweep25,sweep100,sweep400,wide_fp32,wide_tf32",
                     help="comma-separated suite entries (also: capacity)")
+    ap.add_argument("--shard", action="store_true",
+                    help="with N > 1: one graph sharded over the ranks by receiver ranges (all-gather of x, "
+                         "reduce-scatter of dx / d_x, all-reduce of the Theta gradients over NCCL; strong "
+                         "scaling) instead of one independent graph per rank")
     ap.add_argument("--oracle-procs", type=int, default=0,
                     help="processes of the CPU oracle baseline (default: the host cores, at most 32)")
     ap.add_argument("--degree", type=float, default=None, help="mean degree of the sweep workload")
@@ -513,6 +517,67 @@ def run_suite(args):
         torch.cuda.synchronize()
 
 
+def run_sharded(args):
+    """One graph (seed 0) over all ranks by receiver ranges: every step runs
+    forward, backward and double backward through the sharded operator,
+    collectives included (strong scaling).  Time = max over ranks."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import equivariant_gnn_tensor_receiver_b200 as T
+    from equivariant_gnn_tensor_receiver_b200.sharded import LibraryOps, ShardedConv
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    c = W.CONFIGS[args.config]
+    rowptr, col, vec = W.graph_for(args.config, 0, args.degree)
+    N, E = len(rowptr) - 1, len(col)
+    plan = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], radial=c["radial"],
+                  radial_params=c["radial_params"], gemm=args.gemm, family=args.family)
+    sc = ShardedConv(rowptr, col, rank, world, None, device=dev)
+    lg = sc.local
+    f32 = torch.float32
+    todev = lambda a: torch.as_tensor(np.ascontiguousarray(a), dtype=f32, device=dev)
+    sc.ops = LibraryOps(plan, todev(vec[lg.edges]))
+    lo, hi = lg.lo, lg.hi
+    x = todev(W.normal((N, plan.dim_in), 10)[lo:hi])
+    th = todev(W.theta(theta_segments(plan.paths, plan.R, args.family), 11))
+    g = todev(W.normal((N, plan.dim_out), 12)[lo:hi])
+    ggx = todev(W.normal((N, plan.dim_in), 13)[lo:hi])
+    ggv = todev(W.normal((E, 3), 14)[lg.edges])
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        sc.forward(x, th)
+        sc.backward(x, th, g)
+        sc.double_backward(x, th, g, ggx, ggv, None)
+
+    barrier = (lambda: dist.barrier()) if world > 1 else (lambda: None)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    ms = time_ms(step, args.steps, flush)
+    ms_max = reduce_over_ranks(ms, "max", world, dev)
+    if rank == 0:
+        line = {"metric": METRIC, "value": E / (ms_max * 1e-3), "unit": "edges/s", "n_gpus": world,
+                "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_max, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": workload(args), "nodes": N, "edges": E, "gemm": args.gemm,
+                           "family": args.family,
+                           "step": "fwd + bwd(dx,dTheta,dvec) + double bwd(gg_x,gg_vec), sharded",
+                           "l2": "256 MiB buffer zeroed before every timed step, outside the events",
+                           "parallelism": f"receiver ranges over {world} ranks: all-gather x, reduce-scatter "
+                                          "dx / d_x, all-reduce dTheta / d_Theta (NCCL)"}}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def run_ours(args):
     import torch
 
@@ -643,6 +708,8 @@ def main():
         run_reference(args)
     elif args.suite:
         run_suite(args)
+    elif args.shard:
+        run_sharded(args)
     else:
         run_ours(args)
 
