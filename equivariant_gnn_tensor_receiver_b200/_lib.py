@@ -21,7 +21,7 @@ TPCONV_ERR_WORKSPACE_TOO_SMALL = 4
 STATUS = {0: "ok", 1: "invalid argument", 2: "bad irreps", 3: "unsupported", 4: "workspace too small",
           5: "CUDA error", 6: "graph invalid", 7: "timeout", 8: "internal"}
 RADIAL = {"gaussian": 0, "bessel": 1}
-GEMM = {"fp32": 0, "tf32": 1, "bf16": 2, "simt": 3}
+GEMM = {"fp32": 0, "tf32": 1, "simt": 3}
 FAMILY = {"full": 0, "channelwise": 1}
 OP_FORWARD, OP_BACKWARD, OP_DOUBLE_BACKWARD, OP_TRANSPOSE = 0, 1, 2, 3
 

@@ -257,7 +257,7 @@ int tpconv_plan_create(tpconv_plan** out, const char* irreps_in, int l_sh_max,
   if (o.radial != TPCONV_RADIAL_GAUSSIAN && o.radial != TPCONV_RADIAL_BESSEL_COS)
     return TPCONV_ERR_INVALID_ARG;
   if (o.gemm < TPCONV_GEMM_FP32 || o.gemm > TPCONV_GEMM_SIMT) return TPCONV_ERR_INVALID_ARG;
-  if (o.gemm == TPCONV_GEMM_BF16) return TPCONV_ERR_UNSUPPORTED;  // reserved, not built
+  if (o.gemm == 2) return TPCONV_ERR_UNSUPPORTED;  // no half-precision operand mode (see tpconv.h)
   if (o.family != TPCONV_FAMILY_FULL && o.family != TPCONV_FAMILY_CHANNELWISE) return TPCONV_ERR_INVALID_ARG;
   if (o.radial == TPCONV_RADIAL_BESSEL_COS && !(o.radial_p0 > 0)) return TPCONV_ERR_INVALID_ARG;
   if (o.radial == TPCONV_RADIAL_GAUSSIAN && !(o.radial_p1 > o.radial_p0)) return TPCONV_ERR_INVALID_ARG;

@@ -75,10 +75,13 @@ extern "C" {
 #define TPCONV_RADIAL_GAUSSIAN 0   /* exp(-((r-mu_k)/D)^2), mu_k = p0 + k D, D = (p1-p0)/(R-1) */
 #define TPCONV_RADIAL_BESSEL_COS 1 /* sqrt(2/p0) sin(k pi r/p0)/r * (cos(pi r/p0)+1)/2, k=1..R, 0 beyond p0 */
 
-/* precision of the node-level Theta contraction (tensor cores) */
+/* precision of the node-level Theta contractions (tensor cores).  The value 2
+ * is not a mode: plan creation rejects it with TPCONV_ERR_UNSUPPORTED.  A
+ * half-precision operand mode would save nothing here: the contractions read
+ * the fp32 node-side state from HBM once either way and are bound by that
+ * read, not by the tensor pipe. */
 #define TPCONV_GEMM_FP32 0 /* fp32 accuracy: 3xTF32 split on tcgen05      */
 #define TPCONV_GEMM_TF32 1 /* single TF32 pass on tcgen05                 */
-#define TPCONV_GEMM_BF16 2 /* reserved: plan creation returns UNSUPPORTED */
 #define TPCONV_GEMM_SIMT 3 /* plain fp32 FFMA (reference-precision mode)  */
 
 /* operator families (tpconv_options.family).  Both follow "Sobek: streaming

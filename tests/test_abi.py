@@ -118,10 +118,18 @@ def test_workspace_independent_of_edges_and_capped(T):
         assert big <= cap * (1 + 4 * 576 / 22016) + theta_ops + partials + (4 << 20)
 
 
-def test_bf16_mixing_is_reported_unsupported(T):
-    with pytest.raises(T.TPConvError) as e:
-        T.Plan("8x0e+8x1o", 2, "8x0e+8x1o", 4, gemm="bf16")
-    assert e.value.status == 3  # TPCONV_ERR_UNSUPPORTED
+def test_half_precision_mixing_is_rejected(T):
+    """The value between the TF32 and SIMT modes names no mode: plan creation
+    reports it unsupported (the Theta contractions are bound by the fp32 state
+    read, so a half-precision operand mode is not provided)."""
+    import ctypes
+    L = T._lib
+    o = L.default_options()
+    o.gemm = 2
+    h = ctypes.c_void_p()
+    st = L.lib().tpconv_plan_create(ctypes.byref(h), b"8x0e+8x1o", 2, b"8x0e+8x1o", 4, ctypes.byref(o))
+    assert st == 3  # TPCONV_ERR_UNSUPPORTED
+    assert "bf16" not in L.GEMM
 
 
 @pytest.mark.parametrize("gemm,per_op", [("fp32", (2, 4, 12)), ("tf32", (1, 2, 6)), ("simt", (0, 0, 0))])

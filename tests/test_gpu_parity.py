@@ -2,7 +2,7 @@
 
 Tolerance: max-norm relative error ||gpu - ref||_inf / ||ref||_inf <= 1e-5 for
 the fp32 path (the operator's stated bar for fp32 arithmetic); 5e-3 when the
-Theta contraction runs with TF32 / BF16 operands.
+Theta contraction runs with TF32 operands.
 """
 
 import numpy as np
