@@ -81,6 +81,10 @@ def parse():
                     help="with N > 1: one graph sharded over the ranks by receiver ranges (all-gather of x, "
                          "reduce-scatter of dx / d_x, all-reduce of the Theta gradients over NCCL; strong "
                          "scaling) instead of one independent graph per rank")
+    ap.add_argument("--parity-sample", type=int, default=0,
+                    help="after the timed steps, check the step's outputs against the oracle on this many sampled "
+                         "receivers (out, d_g), senders (dx, d_x) and edges (dvec, d_vec), and dTheta / d_Theta "
+                         "by additivity over two receiver halves of the graph; prints a second JSON line")
     ap.add_argument("--oracle-procs", type=int, default=0,
                     help="processes of the CPU oracle baseline (default: the host cores, at most 32)")
     ap.add_argument("--degree", type=float, default=None, help="mean degree of the sweep workload")
@@ -303,6 +307,155 @@ def parallel_oracle(cfg, family, procs, n_recv, warmup, steps):
                       f"{steps} timed steps"}
 
 
+def _sub_problem(rowptr, col, edges):
+    """The listed edges (CSR positions) as a graph of their own: local receivers
+    (sorted) first, then senders that are not receivers; returns
+    (rowptr, col, receivers' global ids, all local nodes' global ids)."""
+    rowptr = np.asarray(rowptr, dtype=np.int64)
+    recv_all = np.repeat(np.arange(len(rowptr) - 1), np.diff(rowptr))
+    edges = np.sort(np.asarray(edges, dtype=np.int64))
+    r = recv_all[edges]
+    s = np.asarray(col, dtype=np.int64)[edges]
+    recvs = np.unique(r)
+    extra = np.setdiff1d(np.unique(s), recvs)
+    nodes = np.concatenate([recvs, extra])
+    pos = {int(g): i for i, g in enumerate(nodes)}
+    lr = np.fromiter((pos[int(v)] for v in r), dtype=np.int64, count=len(r))
+    lc = np.fromiter((pos[int(v)] for v in s), dtype=np.int64, count=len(s))
+    order = np.argsort(lr, kind="stable")
+    lrp = np.concatenate([[0], np.cumsum(np.bincount(lr, minlength=len(nodes)))])
+    return lrp, lc[order], edges[order], recvs, nodes
+
+
+def _parity_worker(job):
+    """One oracle job of the parity check: (kind, config, family, arrays) -> arrays."""
+    kind, cfg, family, a = job
+    from oracle import conv
+    c = W.CONFIGS[cfg]
+    prob = conv.Problem(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], c["radial"],
+                        tuple(c["radial_params"]), family=family)
+    rp, col, vec, x, th, g = a["rowptr"], a["col"], a["vec"], a["x"], a["theta"], a["g"]
+    if kind == "recv":
+        out = conv.forward(prob, rp, col, vec, x, th)
+        return {"out": out}
+    if kind == "recv_dbl":
+        r = conv.double_backward(prob, rp, col, vec, x, th, g, a["gg_x"], a["gg_vec"], None)
+        return {"d_g": r["d_g"]}
+    if kind == "send":
+        return {"dx": conv.backward(prob, rp, col, vec, x, th, g)["dx"]}
+    if kind == "send_dbl":
+        r = conv.double_backward(prob, rp, col, vec, x, th, g, a["gg_x"], a["gg_vec"], None)
+        return {"d_x": r["d_x"]}
+    if kind == "edge":
+        rb = conv.backward(prob, rp, col, vec, x, th, g)
+        r = conv.double_backward(prob, rp, col, vec, x, th, g, a["gg_x"], a["gg_vec"], None)
+        return {"dvec": rb["dvec"], "d_vec": r["d_vec"]}
+    raise ValueError(kind)
+
+
+def parity_check(args, work, graph, procs, k):
+    """Sampled parity of one full step of the workload against the oracle (see --parity-sample)."""
+    import multiprocessing as mp
+    import torch
+    rowptr, col, vec = graph
+    N, E = work.N, work.E
+    h = {key: v.numpy() for key, v in work.host.items()}
+    f64 = lambda a: np.asarray(a, dtype=np.float32).astype(np.float64)
+    x, th, g, ggx, ggv, v32 = (f64(h[key]) for key in ("x", "theta", "g", "gg_x", "gg_vec", "vec"))
+    gpu = {key: t.double().cpu().numpy() for key, t in work.outs.items()}
+    rng = np.random.default_rng(12345)
+    recv_all = np.repeat(np.arange(N), np.diff(np.asarray(rowptr, dtype=np.int64)))
+    k_dbl = max(1, k // 4)
+    rs = np.sort(rng.choice(N, k, replace=False))
+    ss = np.sort(rng.choice(N, k, replace=False))
+    es = np.sort(rng.choice(E, k, replace=False))
+    col64 = np.asarray(col, dtype=np.int64)
+    rp64 = np.asarray(rowptr, dtype=np.int64)
+
+    def job(kind, edges):
+        lrp, lc, eids, recvs, nodes = _sub_problem(rowptr, col, edges)
+        a = {"rowptr": lrp, "col": lc, "vec": v32[eids], "x": x[nodes], "theta": th,
+             "g": g[nodes], "gg_x": ggx[nodes], "gg_vec": ggv[eids]}
+        return (kind, args.config, args.family, a), (recvs, nodes, eids)
+
+    def edges_of_recv(r):
+        return np.concatenate([np.arange(rp64[i], rp64[i + 1]) for i in r]) if len(r) else np.zeros(0, np.int64)
+
+    def edges_of_send(sn):
+        return np.nonzero(np.isin(col64, sn))[0]
+
+    split = lambda arr, n: [a for a in np.array_split(arr, n) if len(a)]
+    jobs, meta = [], []
+    for part in split(rs, procs):
+        j, m = job("recv", edges_of_recv(part)); jobs.append(j); meta.append(("recv", part, m))
+    for part in split(rs[:k_dbl], procs):
+        j, m = job("recv_dbl", edges_of_recv(part)); jobs.append(j); meta.append(("recv_dbl", part, m))
+    for part in split(ss, procs):
+        j, m = job("send", edges_of_send(part)); jobs.append(j); meta.append(("send", part, m))
+    for part in split(ss[:k_dbl], procs):
+        j, m = job("send_dbl", edges_of_send(part)); jobs.append(j); meta.append(("send_dbl", part, m))
+    for part in split(es, procs):
+        j, m = job("edge", part); jobs.append(j); meta.append(("edge", part, m))
+    env = {key: os.environ.get(key) for key in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+    for key in env:
+        os.environ[key] = "1"
+    t0 = time.perf_counter()
+    try:
+        with mp.get_context("spawn").Pool(procs) as pool:
+            results = pool.map(_parity_worker, jobs, chunksize=1)
+    finally:
+        for key, v in env.items():
+            if v is None:
+                os.environ.pop(key, None)
+            else:
+                os.environ[key] = v
+    ref = {key: [] for key in ("out", "d_g", "dx", "d_x", "dvec", "d_vec")}
+    got = {key: [] for key in ref}
+    for (kind, part, (recvs, nodes, eids)), res in zip(meta, results):
+        pos = {int(v): i for i, v in enumerate(nodes)}
+        rows = np.array([pos[int(v)] for v in part])
+        if kind in ("recv", "recv_dbl", "send", "send_dbl"):
+            key = {"recv": "out", "recv_dbl": "d_g", "send": "dx", "send_dbl": "d_x"}[kind]
+            ref[key].append(res[key][rows])
+            got[key].append(gpu[key][part])
+        else:
+            order = np.argsort(eids)  # back to the sampled (sorted) edge order
+            for key in ("dvec", "d_vec"):
+                ref[key].append(res[key][order])
+                got[key].append(gpu[key][np.sort(eids)])
+    errs = {}
+    for key in ref:
+        rr, gg = np.concatenate(ref[key]), np.concatenate(got[key])
+        errs[key] = float(np.abs(gg - rr).max() / max(np.abs(rr).max(), 1e-30))
+    # dTheta and d_Theta: the full graph against the sum over its two receiver
+    # halves (the library on both sides; additivity holds at any size)
+    T = work.T
+    half = N // 2
+    sums = {}
+    d = work.d
+    for lo, hi in ((0, half), (half, N)):
+        sub_rp = np.concatenate([np.zeros(lo, np.int64), rp64[lo:hi + 1] - rp64[lo],
+                                 np.full(N - hi, rp64[hi] - rp64[lo], np.int64)])
+        e0, e1 = int(rp64[lo]), int(rp64[hi])
+        Gs = T.Graph(torch.as_tensor(sub_rp, dtype=torch.int32, device=work.dev), d["col"][e0:e1],
+                     d["vec"][e0:e1])
+        a = T.backward(work.plan, Gs, d["x"], d["theta"], d["g"], want=("dtheta",))["dtheta"]
+        b = T.double_backward(work.plan, Gs, d["x"], d["theta"], d["g"], d["gg_x"], d["gg_vec"][e0:e1], None,
+                              want=("d_theta",))["d_theta"]
+        torch.cuda.synchronize()
+        sums["dtheta"] = sums.get("dtheta", 0.0) + a.double().cpu().numpy()
+        sums["d_theta"] = sums.get("d_theta", 0.0) + b.double().cpu().numpy()
+        del Gs, a, b
+        torch.cuda.empty_cache()
+    for key in ("dtheta", "d_theta"):
+        errs[key + "_additivity"] = float(np.abs(sums[key] - gpu[key]).max() / max(np.abs(gpu[key]).max(), 1e-30))
+    tol = 1e-5 if args.gemm in ("fp32", "simt") else 5e-3
+    return {"parity": args.config, "gemm": args.gemm, "family": args.family, "nodes": N, "edges": E,
+            "sampled_receivers": k, "sampled_senders": k, "sampled_edges": k, "sampled_dbl_nodes": k_dbl,
+            "max_norm_rel_err": errs, "tolerance": tol, "pass": all(v < tol for v in errs.values()),
+            "oracle_s": round(time.perf_counter() - t0, 1), "oracle_procs": procs}
+
+
 def reduce_over_ranks(v, op, world, device):
     """Max or sum of a per-rank scalar over the default process group (any
     backend: nccl with a CUDA device, gloo with the CPU); identity at world 1."""
@@ -346,7 +499,7 @@ class Work:
     def __init__(self, T, L, config, graph, gemm, family, cap, dev, seed=0):
         import torch
         c = W.CONFIGS[config]
-        self.L, self.dev = L, dev
+        self.T, self.L, self.dev, self.cap = T, L, dev, cap
         rowptr, col, vec = graph
         self.N, self.E = N, E = len(rowptr) - 1, len(col)
         self.plan = plan = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], radial=c["radial"],
@@ -697,6 +850,11 @@ def run_ours(args):
             "library_static_bytes": L.static_device_bytes(),
         }
         print(json.dumps(line), flush=True)
+    if args.parity_sample and world == 1:
+        work.step()  # outputs of one step over the resident inputs
+        torch.cuda.synchronize()
+        procs = args.oracle_procs or min(32, host_cores())
+        print(json.dumps(parity_check(args, work, graph, procs, args.parity_sample)), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

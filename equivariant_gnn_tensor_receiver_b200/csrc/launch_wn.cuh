@@ -1,26 +1,13 @@
-// Launchers of the warp-per-node edge streams (instantiated per (RM, LF[, CPL])
-// in tu_wn_*.cu).  One warp per node of the chunk, kWnWarps nodes per CTA.
+// Launchers of the channel-lane warp-per-node edge streams (instantiated per
+// (RM, LF[, CPL]) in tu_wn_{fwd,send,dbla,dbls}_*.cu).  One warp per node of the
+// chunk, kWnWarps nodes per CTA.
 #pragma once
 
 #include "launch_streams.cuh"
-#include "launchers.h"
+#include "launch_wn_common.cuh"
 #include "streams_wn.cuh"
-#include "streams_wna.cuh"
 
 namespace tpc {
-
-// path-major grid of the first pieces (channel-lane streams)
-inline unsigned wn_grid_pm(const DevPlan& d, int nc) { return unsigned(d.P) * unsigned((nc + kWnWarps - 1) / kWnWarps); }
-// persistent grid: as many CTAs as fit on the device at once
-template <class K>
-unsigned wn_grid(K kernel, int smem) {
-  int dev = 0, sms = 148, per = 1;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kernel, 32 * kWnWarps, smem) != cudaSuccess || per < 1)
-    per = 1;
-  return unsigned(sms * per);
-}
 
 template <int RM, int LF, int CPL, bool RECV, bool DBL>
 cudaError_t wn_smem(int bytes) {
@@ -33,17 +20,6 @@ cudaError_t wn_smem(int bytes) {
   }
   return e;
 }
-template <int RM, int LF, bool DBL>
-cudaError_t wna_smem(int bytes) {
-  cudaError_t e = cudaFuncSetAttribute(k_wn_adj<RM, LF, DBL, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       bytes);
-  if constexpr (DBL) {
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(k_wn_adj<RM, LF, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  }
-  return e;
-}
-
 template <int RM, int LF, int CPL>
 cudaError_t launch_wn_fwd(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,
                           const float* x, float* A, const int* extra, int* counter, int seg, cudaStream_t st) {
@@ -117,36 +93,8 @@ cudaError_t launch_wn_dbls(const DevPlan& d, int s0, int nc, const int* s_rowptr
   return cudaGetLastError();
 }
 
-template <int RM, int LF>
-cudaError_t launch_wn_adj(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,
-                          const float* x, const float* G, float* dvec, float* dY, float* db, const int* extra,
-                          int* counter, cudaStream_t st) {
-  if (nc <= 0) return cudaSuccess;
-  auto k = k_wn_adj<RM, LF, false, false>;
-  k<<<wn_grid(k, d.wn_smem_adj), 32 * kWnWarps, d.wn_smem_adj, st>>>(d, r0, nc, rowptr, col, vec, nullptr, x, nullptr,
-                                                                      G, nullptr, dvec, dY, db, extra, counter);
-  return cudaGetLastError();
-}
-
-template <int RM, int LF>
-cudaError_t launch_wn_dadj(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,
-                           const float* ggv, const float* x, const float* ggx, const float* G, const float* Gt,
-                           float* dvec, const int* extra, int* counter, cudaStream_t st) {
-  if (nc <= 0) return cudaSuccess;
-  if (Gt) {
-    auto k = k_wn_adj<RM, LF, true, true>;
-    k<<<wn_grid(k, d.wn_smem_dadj), 32 * kWnWarps, d.wn_smem_dadj, st>>>(d, r0, nc, rowptr, col, vec, ggv, x, ggx, G,
-                                                                          Gt, dvec, nullptr, nullptr, extra, counter);
-  } else {
-    auto k = k_wn_adj<RM, LF, true, false>;
-    k<<<wn_grid(k, d.wn_smem_dadj), 32 * kWnWarps, d.wn_smem_dadj, st>>>(d, r0, nc, rowptr, col, vec, ggv, x, ggx, G,
-                                                                          nullptr, dvec, nullptr, nullptr, extra,
-                                                                          counter);
-  }
-  return cudaGetLastError();
-}
-
 }  // namespace tpc
+
 
 // One translation unit per kernel instantiation keeps the parallel build even.
 #define TPC_WN_TU_CPL(tag, form, RM, LF, CPL, RECV, DBL, ...)                 \
@@ -159,8 +107,3 @@ cudaError_t launch_wn_dadj(const DevPlan& d, int r0, int nc, const int* rowptr, 
   template cudaError_t launch_wn_##form<RM, LF>(__VA_ARGS__);                 \
   }                                                                           \
   TPC_REGISTER_TU(tag, (&tpc::wn_smem<RM, LF, 1, RECV, DBL>))
-#define TPC_WNA_TU(tag, form, RM, LF, DBL, ...)                               \
-  namespace tpc {                                                             \
-  template cudaError_t launch_wn_##form<RM, LF>(__VA_ARGS__);                 \
-  }                                                                           \
-  TPC_REGISTER_TU(tag, (&tpc::wna_smem<RM, LF, DBL>))

@@ -1,0 +1,57 @@
+// Launchers of the edge-lane (receiver adjoint) warp-per-node streams
+// (instantiated per (RM, LF) in tu_wn_{adj,dadj}_*.cu).
+#pragma once
+
+#include "launch_streams.cuh"
+#include "launch_wn_common.cuh"
+#include "streams_wna.cuh"
+
+namespace tpc {
+
+template <int RM, int LF, bool DBL>
+cudaError_t wna_smem(int bytes) {
+  cudaError_t e = cudaFuncSetAttribute(k_wn_adj<RM, LF, DBL, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       bytes);
+  if constexpr (DBL) {
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_wn_adj<RM, LF, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  }
+  return e;
+}
+
+template <int RM, int LF>
+cudaError_t launch_wn_adj(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,
+                          const float* x, const float* G, float* dvec, float* dY, float* db, const int* extra,
+                          int* counter, cudaStream_t st) {
+  if (nc <= 0) return cudaSuccess;
+  auto k = k_wn_adj<RM, LF, false, false>;
+  k<<<wn_grid(k, d.wn_smem_adj), 32 * kWnWarps, d.wn_smem_adj, st>>>(d, r0, nc, rowptr, col, vec, nullptr, x, nullptr,
+                                                                      G, nullptr, dvec, dY, db, extra, counter);
+  return cudaGetLastError();
+}
+
+template <int RM, int LF>
+cudaError_t launch_wn_dadj(const DevPlan& d, int r0, int nc, const int* rowptr, const int* col, const float* vec,
+                           const float* ggv, const float* x, const float* ggx, const float* G, const float* Gt,
+                           float* dvec, const int* extra, int* counter, cudaStream_t st) {
+  if (nc <= 0) return cudaSuccess;
+  if (Gt) {
+    auto k = k_wn_adj<RM, LF, true, true>;
+    k<<<wn_grid(k, d.wn_smem_dadj), 32 * kWnWarps, d.wn_smem_dadj, st>>>(d, r0, nc, rowptr, col, vec, ggv, x, ggx, G,
+                                                                          Gt, dvec, nullptr, nullptr, extra, counter);
+  } else {
+    auto k = k_wn_adj<RM, LF, true, false>;
+    k<<<wn_grid(k, d.wn_smem_dadj), 32 * kWnWarps, d.wn_smem_dadj, st>>>(d, r0, nc, rowptr, col, vec, ggv, x, ggx, G,
+                                                                          nullptr, dvec, nullptr, nullptr, extra,
+                                                                          counter);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace tpc
+
+#define TPC_WNA_TU(tag, form, RM, LF, DBL, ...)                               \
+  namespace tpc {                                                             \
+  template cudaError_t launch_wn_##form<RM, LF>(__VA_ARGS__);                 \
+  }                                                                           \
+  TPC_REGISTER_TU(tag, (&tpc::wna_smem<RM, LF, DBL>))

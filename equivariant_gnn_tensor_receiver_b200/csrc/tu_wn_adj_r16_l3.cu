@@ -1,4 +1,4 @@
 // Warp-per-node stream (receiver adjoint, first order), radial width 16, feature degrees <= 3.
-#include "launch_wn.cuh"
+#include "launch_wn_adj.cuh"
 
 TPC_WNA_TU(wn_adj_r16_l3, adj, 16, 3, false, const DevPlan&, int, int, const int*, const int*, const float*, const float*, const float*, float*, float*, float*, const int*, int*, cudaStream_t)

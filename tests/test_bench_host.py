@@ -1,0 +1,67 @@
+"""Host logic of the benchmark's sampled parity check (no GPU): the oracle on
+the sub-problem that the check builds for sampled receivers, senders and edges
+reproduces the oracle on the whole graph for exactly those rows."""
+
+import importlib.util
+import os
+
+import numpy as np
+
+import workloads as W
+from oracle import conv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench", os.path.join(ROOT, "bench.py"))
+    m = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(m)
+    return m
+
+
+def test_sub_problems_reproduce_the_whole_graph():
+    B = _bench()
+    c = W.CONFIGS["tiny"]
+    prob = conv.Problem(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], c["radial"], c["radial_params"])
+    rowptr, col, vec = W.graph_for("tiny", 2)
+    N, E = len(rowptr) - 1, len(col)
+    x, g = W.normal((N, prob.dim_in), 1), W.normal((N, prob.dim_out), 2)
+    th = W.theta([(c["R"] * p.c_in * p.c_out, 0.2) for p in prob.paths], 3)
+    ggx, ggv = W.normal((N, prob.dim_in), 4), W.normal((E, 3), 5)
+    full_f = conv.forward(prob, rowptr, col, vec, x, th)
+    full_b = conv.backward(prob, rowptr, col, vec, x, th, g)
+    full_d = conv.double_backward(prob, rowptr, col, vec, x, th, g, ggx, ggv, None)
+    rp = np.asarray(rowptr, dtype=np.int64)
+    rs = np.array([3, 17, 40])
+    edges = np.concatenate([np.arange(rp[i], rp[i + 1]) for i in rs])
+    lrp, lc, eids, recvs, nodes = B._sub_problem(rowptr, col, edges)
+    assert np.array_equal(np.sort(eids), np.sort(edges)) and np.array_equal(recvs, rs)
+    pos = {int(v): i for i, v in enumerate(nodes)}
+    rows = [pos[int(r)] for r in rs]
+    a = {"rowptr": lrp, "col": lc, "vec": vec[eids], "x": x[nodes], "theta": th, "g": g[nodes],
+         "gg_x": ggx[nodes], "gg_vec": ggv[eids]}
+    out = B._parity_worker(("recv", "tiny", "full", a))["out"]
+    assert np.allclose(out[rows], full_f[rs], rtol=0, atol=1e-12)
+    d_g = B._parity_worker(("recv_dbl", "tiny", "full", a))["d_g"]
+    assert np.allclose(d_g[rows], full_d["d_g"][rs], rtol=0, atol=1e-11)
+    # senders: all their out-edges
+    ss = np.array([5, 30])
+    es = np.nonzero(np.isin(col, ss))[0]
+    lrp, lc, eids, recvs, nodes = B._sub_problem(rowptr, col, es)
+    pos = {int(v): i for i, v in enumerate(nodes)}
+    a = {"rowptr": lrp, "col": lc, "vec": vec[eids], "x": x[nodes], "theta": th, "g": g[nodes],
+         "gg_x": ggx[nodes], "gg_vec": ggv[eids]}
+    rows = [pos[int(s)] for s in ss]
+    assert np.allclose(B._parity_worker(("send", "tiny", "full", a))["dx"][rows], full_b["dx"][ss], atol=1e-11)
+    assert np.allclose(B._parity_worker(("send_dbl", "tiny", "full", a))["d_x"][rows], full_d["d_x"][ss],
+                       atol=1e-10)
+    # single edges
+    ee = np.array([0, 77, 300, 511])
+    lrp, lc, eids, recvs, nodes = B._sub_problem(rowptr, col, ee)
+    a = {"rowptr": lrp, "col": lc, "vec": vec[eids], "x": x[nodes], "theta": th, "g": g[nodes],
+         "gg_x": ggx[nodes], "gg_vec": ggv[eids]}
+    r = B._parity_worker(("edge", "tiny", "full", a))
+    order = np.argsort(eids)
+    assert np.allclose(r["dvec"][order], full_b["dvec"][np.sort(eids)], atol=1e-11)
+    assert np.allclose(r["d_vec"][order], full_d["d_vec"][np.sort(eids)], atol=1e-10)
