@@ -87,22 +87,13 @@ struct __align__(64) DtParams {
   uint64_t wait_ns;
 };
 
-// Shared memory: as the Theta contractions' GEMM.  3xTF32: a ring of raw A
-// tiles (TMA -> converter, returned as soon as they are split) and a small
-// ring of operand stages (A hi, A lo, B hi, B lo) for the MMAs; TF32: one ring
-// of (A, B) stages.
-template <int BN, bool SPLIT>
+template <int BN>
 struct DtSmem {
   static constexpr int kA = kBM * kBK * 4;  // 16 KB: four 32 x 32 boxes
   static constexpr int kB = BN * kBK * 4;
-  static constexpr int kBudget = 192 * 1024;
-  static constexpr int kOpStage = SPLIT ? 2 * kA + 2 * kB : kA + kB;
-  static constexpr int kOps0 = SPLIT ? (2 * kOpStage + 2 * kA <= kBudget ? 2 : 1) : kBudget / kOpStage;
-  static constexpr int kOps = kOps0 > 8 ? 8 : kOps0;
-  static constexpr int kRaw0 = SPLIT ? (kBudget - kOps * kOpStage) / kA : 0;
-  static constexpr int kRaw = kRaw0 > 8 ? 8 : kRaw0;
-  static constexpr int kBytes = kRaw * kA + kOps * kOpStage + 1024 + 512;
-  static_assert(!SPLIT || kRaw >= 2, "the raw ring needs two stages");
+  static constexpr int kStage = 2 * kA + 2 * kB;
+  static constexpr int kStages = (200 * 1024) / kStage >= 4 ? 4 : ((200 * 1024) / kStage >= 3 ? 3 : 2);
+  static constexpr int kBytes = kStages * kStage + 1024 + 256;
 };
 
 // TMEM accumulators; 3xTF32 with column tiles of at most 128 runs the round
@@ -125,8 +116,8 @@ __device__ __forceinline__ bool waitp(uint64_t* b, uint32_t parity, uint64_t lim
 
 template <int BN, bool SPLIT>
 __global__ void __launch_bounds__(192, 1) k_dtheta_tc(const __grid_constant__ DtParams P) {
-  using SM = DtSmem<BN, SPLIT>;
-  constexpr int SR = SM::kRaw, SO = SM::kOps;
+  using SM = DtSmem<BN>;
+  constexpr int S = SM::kStages;
   constexpr uint32_t kCols = DtAcc<BN, SPLIT>::kCols;
   constexpr int NACC = DtAcc<BN, SPLIT>::N;
   constexpr uint32_t kAlloc = DtAcc<BN, SPLIT>::kAlloc;
@@ -135,14 +126,10 @@ __global__ void __launch_bounds__(192, 1) k_dtheta_tc(const __grid_constant__ Dt
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* raw_base = base;               // SR raw A tiles
-  unsigned char* op_base = base + SR * SM::kA;  // SO operand stages
-  uint64_t* rawfull = reinterpret_cast<uint64_t*>(op_base + SO * SM::kOpStage);
-  uint64_t* rawfree = rawfull + 8;
-  uint64_t* opfull = rawfree + 8;   // TMA of the stage's B halves (TF32: of A and B)
-  uint64_t* opconv = opfull + 8;    // the converter wrote the stage's A halves
-  uint64_t* opfree = opconv + 8;    // the stage's MMAs completed
-  uint64_t* accf = opfree + 8;
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + S * SM::kStage);
+  uint64_t* conv = full + S;
+  uint64_t* empty = conv + S;
+  uint64_t* accf = empty + S;
   uint64_t* bfull = accf + 1;   // [2] a round of the bank is complete
   uint64_t* bfree = bfull + 2;  // [2] the bank has been added into registers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bfree + 2);
@@ -163,14 +150,10 @@ __global__ void __launch_bounds__(192, 1) k_dtheta_tc(const __grid_constant__ Dt
   const uint64_t limit = P.wait_ns;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SR; ++s) {
-      mbar_init(&rawfull[s], 1);
-      mbar_init(&rawfree[s], 128);
-    }
-    for (int s = 0; s < SO; ++s) {
-      mbar_init(&opfull[s], 1);
-      mbar_init(&opconv[s], 128);
-      mbar_init(&opfree[s], 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&conv[s], 128);
+      mbar_init(&empty[s], 1);
     }
     mbar_init(accf, 1);
     for (int b = 0; b < 2; ++b) {
@@ -186,55 +169,45 @@ __global__ void __launch_bounds__(192, 1) k_dtheta_tc(const __grid_constant__ Dt
   fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  auto sRaw = [&](int r) { return raw_base + r * SM::kA; };
-  auto sA = [&](int c) { return op_base + c * SM::kOpStage; };
-  auto sAlo = [&](int c) { return op_base + c * SM::kOpStage + SM::kA; };
-  auto sB = [&](int c) { return op_base + c * SM::kOpStage + (SPLIT ? 2 : 1) * SM::kA; };
-  auto sBlo = [&](int c) { return op_base + c * SM::kOpStage + 2 * SM::kA + SM::kB; };
+  auto sA = [&](int s) { return base + s * SM::kStage; };
+  auto sAlo = [&](int s) { return base + s * SM::kStage + SM::kA; };
+  auto sB = [&](int s) { return base + s * SM::kStage + 2 * SM::kA; };
+  auto sBlo = [&](int s) { return base + s * SM::kStage + 2 * SM::kA + SM::kB; };
 
-  int issued = 0;  // K steps whose loads this producer lane issued
-  if (warp == 0 && lane < (SPLIT ? 2 : 1)) {
-    // lane 0: A tiles (3xTF32: into the raw ring); lane 1 (3xTF32): B halves into the operand stages
-    const CUtensorMap* ma = &P.a[G.map];
-    const CUtensorMap* mbh = &P.bh[G.map];
-    const CUtensorMap* mbl = &P.bl[G.map];
-    const bool into_raw = SPLIT && lane == 0;
-    const int S = into_raw ? SR : SO;
-    for (int kt = 0; kt < nk; ++kt) {
-      const int s = kt % S;
-      uint64_t* freeb = into_raw ? &rawfree[s] : &opfree[s];
-      if (kt >= S && !waitp(freeb, ((kt / S) + 1) & 1, limit, 1)) {
-        *abort_flag = 1;
-        break;
-      }
-      if (*abort_flag) break;
-      const int kr = k0 + kt * kBK;
-      if (into_raw || !SPLIT) {
-        unsigned char* dA = into_raw ? sRaw(s) : sA(s);
-        uint64_t* bar = into_raw ? &rawfull[s] : &opfull[s];
-        mbar_expect_tx(bar, SM::kA + (SPLIT ? 0 : SM::kB));
+  int issued = 0;
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t bytes = SM::kA + (SPLIT ? 2 : 1) * SM::kB;
+      const CUtensorMap* ma = &P.a[G.map];
+      const CUtensorMap* mbh = &P.bh[G.map];
+      const CUtensorMap* mbl = &P.bl[G.map];
+      for (int kt = 0; kt < nk; ++kt) {
+        const int s = kt % S;
+        if (kt >= S && !waitp(&empty[s], ((kt / S) + 1) & 1, limit, 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        if (*abort_flag) break;
+        const int kr = k0 + kt * kBK;
+        mbar_expect_tx(&full[s], bytes);
 #pragma unroll
-        for (int j = 0; j < kBM / 32; ++j) tma_load_2d(dA + j * 4096, ma, bar, mcol + 32 * j, kr);
-        if (!SPLIT) tma_load_2d(sB(s), mbh, bar, kr, 0);
-      } else {
-        mbar_expect_tx(&opfull[s], 2 * SM::kB);
-        tma_load_2d(sB(s), mbh, &opfull[s], kr, 0);
-        tma_load_2d(sBlo(s), mbl, &opfull[s], kr, 0);
+        for (int j = 0; j < kBM / 32; ++j) tma_load_2d(sA(s) + j * 4096, ma, &full[s], mcol + 32 * j, kr);
+        tma_load_2d(sB(s), mbh, &full[s], kr, 0);
+        if (SPLIT) tma_load_2d(sBlo(s), mbl, &full[s], kr, 0);
+        issued = kt + 1;
       }
-      issued = kt + 1;
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_tf32(kBM, BN, /*a_mn=*/true, /*b_mn=*/false);
       for (int kt = 0; kt < nk; ++kt) {
-        const int s = kt % SO;
-        const uint32_t par = (kt / SO) & 1;
+        const int s = kt % S;
         const int r = DRAIN ? kt / RS::D : 0, j = DRAIN ? kt - r * RS::D : kt, bank = r & 1;
         if (DRAIN && j == 0 && r >= 2 && !waitp(&bfree[bank], ((r >> 1) - 1) & 1, limit, 7)) {
           *abort_flag = 1;
           break;
         }
-        if (!waitp(&opfull[s], par, limit, 2) || (SPLIT && !waitp(&opconv[s], par, limit, 2)) || *abort_flag) {
+        if (!waitp(SPLIT ? &conv[s] : &full[s], (kt / S) & 1, limit, 2) || *abort_flag) {
           *abort_flag = 1;
           break;
         }
@@ -255,12 +228,12 @@ __global__ void __launch_bounds__(192, 1) k_dtheta_tc(const __grid_constant__ Dt
             mma_tf32(td, sw128b32_mn_desc(al + kk * 1024, 4096, 512), db, idesc, 1u);
           }
         }
-        mma_commit(&opfree[s]);
+        mma_commit(&empty[s]);
         if (DRAIN && (j == RS::D - 1 || kt == nk - 1)) mma_commit(&bfull[bank]);
       }
       mma_commit(accf);  // fires once every MMA issued above has completed
     }
-  } else if (warp >= 2) {
+  } else {
     // warps 2..5: split A (3xTF32), add finished rounds into registers, store
     // the partial tile; exit decisions are warp-uniform (TMEM loads are
     // warp-collective)
@@ -281,28 +254,19 @@ __global__ void __launch_bounds__(192, 1) k_dtheta_tc(const __grid_constant__ Dt
       ++drained;
       return true;
     };
-    if constexpr (SPLIT) {
+    if (SPLIT) {
       for (int kt = 0; kt < nk; ++kt) {
-        const int r = kt % SR, s = kt % SO;
-        const bool got = waitp(&rawfull[r], (kt / SR) & 1, limit, 3) &&
-                         (kt < SO || waitp(&opfree[s], ((kt / SO) + 1) & 1, limit, 3)) && !*abort_flag;
-        if (!__all_sync(0xffffffffu, got)) {
+        const int s = kt % S;
+        if (!__all_sync(0xffffffffu, waitp(&full[s], (kt / S) & 1, limit, 3) && !*abort_flag)) {
           *abort_flag = 1;
           break;
         }
-        // elementwise split: the raw tile and the halves share the swizzled layout
-        const float4* r4 = reinterpret_cast<const float4*>(sRaw(r));
         float4* a4 = reinterpret_cast<float4*>(sA(s));
         float4* l4 = reinterpret_cast<float4*>(sAlo(s));
 #pragma unroll 4
-        for (int i = t; i < kBM * kBK / 4; i += 128) {
-          a4[i] = r4[i];
-          split4(a4 + i, l4 + i);
-        }
-        // the MMAs (async proxy) read the halves; TMA may refill the raw tile
+        for (int i = t; i < kBM * kBK / 4; i += 128) split4(a4 + i, l4 + i);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive(&opconv[s]);
-        mbar_arrive(&rawfree[r]);
+        mbar_arrive(&conv[s]);
         if constexpr (DRAIN) {
           const int rr = RS::drain_after(kt);
           if (rr >= 0 && !drain(rr)) {
@@ -344,11 +308,9 @@ __global__ void __launch_bounds__(192, 1) k_dtheta_tc(const __grid_constant__ Dt
     }
   }
   // before exit: no copy and no MMA of this CTA may still be in flight
-  if (warp == 0 && lane < (SPLIT ? 2 : 1) && *abort_flag) {
-    const bool into_raw = SPLIT && lane == 0;
-    const int S = into_raw ? SR : SO;
+  if (warp == 0 && lane == 0 && *abort_flag) {
     for (int kt = (issued > S ? issued - S : 0); kt < issued; ++kt)
-      waitp(into_raw ? &rawfull[kt % S] : &opfull[kt % S], (kt / S) & 1, kDrainLimitNs, 5);
+      waitp(&full[kt % S], (kt / S) & 1, kDrainLimitNs, 5);
   }
   if (warp == 1 && lane == 0) waitp(accf, 0, kDrainLimitNs, 6);
   fence_before_sync();
@@ -469,12 +431,12 @@ int64_t kpad_of(int nc, int n1) { return (int64_t(nc) * n1 + 3) & ~int64_t(3); }
 template <int BN, bool SPLIT>
 cudaError_t set_smem() {
   return cudaFuncSetAttribute(k_dtheta_tc<BN, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              DtSmem<BN, SPLIT>::kBytes);
+                              DtSmem<BN>::kBytes);
 }
 
 template <int BN, bool SPLIT>
 cudaError_t launch(const DtParams& p, int n_cta, cudaStream_t st) {
-  k_dtheta_tc<BN, SPLIT><<<n_cta, 192, DtSmem<BN, SPLIT>::kBytes, st>>>(p);
+  k_dtheta_tc<BN, SPLIT><<<n_cta, 192, DtSmem<BN>::kBytes, st>>>(p);
   return cudaGetLastError();
 }
 

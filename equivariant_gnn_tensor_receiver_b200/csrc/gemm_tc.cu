@@ -54,23 +54,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, uint64_t
   return false;
 }
 
-// Shared memory.  3xTF32: raw A tiles have a ring of their own (TMA -> the
-// converter warps), and a small ring of operand stages (A hi, A lo, B hi, B lo)
-// feeds the MMAs; a raw tile returns to TMA as soon as it has been split, so
-// up to kRaw tiles of A are in flight whatever the MMA is doing.  TF32: one
-// ring of (A, B) stages read by the MMAs directly.
-template <int BN, bool SPLIT>
+template <int BN>
 struct TcSmem {
-  static constexpr int kA = kBM * kBK * 4;  // 16 KB
-  static constexpr int kB = BN * kBK * 4;   // BN x 128 B
-  static constexpr int kBudget = 192 * 1024;
-  static constexpr int kOpStage = SPLIT ? 2 * kA + 2 * kB : kA + kB;
-  static constexpr int kOps0 = SPLIT ? (2 * kOpStage + 2 * kA <= kBudget ? 2 : 1) : kBudget / kOpStage;
-  static constexpr int kOps = kOps0 > 8 ? 8 : kOps0;
-  static constexpr int kRaw0 = SPLIT ? (kBudget - kOps * kOpStage) / kA : 0;
-  static constexpr int kRaw = kRaw0 > 8 ? 8 : kRaw0;
-  static constexpr int kBytes = kRaw * kA + kOps * kOpStage + 1024 /*align*/ + 512 /*barriers, slot, flag*/;
-  static_assert(!SPLIT || kRaw >= 2, "the raw ring needs two stages");
+  static constexpr int kA = kBM * kBK * 4;   // 16 KB
+  static constexpr int kB = BN * kBK * 4;    // BN x 128 B
+  static constexpr int kStage = 2 * kA + 2 * kB;
+  static constexpr int kStages = (200 * 1024) / kStage >= 4 ? 4 : ((200 * 1024) / kStage >= 3 ? 3 : 2);
+  static constexpr int kBytes = kStages * kStage + 1024 /*align*/ + 256 /*barriers: 3 x stages + 5, slot, flag*/;
 };
 
 // Accumulators in TMEM.  The 3xTF32 mode uses NACC of them in the round
@@ -90,27 +80,22 @@ __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmBlo, int M, int N, int K, TcOut out, int accumulate,
               uint64_t limit) {
-  using SM = TcSmem<BN, SPLIT>;
-  constexpr int SR = SM::kRaw, SO = SM::kOps;
+  using SM = TcSmem<BN>;
+  constexpr int S = SM::kStages;
   constexpr uint32_t kCols = TcAcc<BN, SPLIT>::kCols;
   constexpr int NACC = TcAcc<BN, SPLIT>::N;
   constexpr uint32_t kAlloc = TcAcc<BN, SPLIT>::kAlloc;
   constexpr bool DRAIN = TcAcc<BN, SPLIT>::kDrain;
   using RS = Rounds<NACC>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* base =
-      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* raw_base = base;                    // SR raw A tiles
-  unsigned char* op_base = base + SR * SM::kA;       // SO operand stages
-  uint64_t* rawfull = reinterpret_cast<uint64_t*>(op_base + SO * SM::kOpStage);
-  uint64_t* rawfree = rawfull + 8;
-  uint64_t* opfull = rawfree + 8;  // TMA of the stage's B halves (TF32: of A and B)
-  uint64_t* opconv = opfull + 8;   // the converter wrote the stage's A halves
-  uint64_t* opfree = opconv + 8;   // the stage's MMAs completed
-  uint64_t* accf = opfree + 8;
-  uint64_t* bankfull = accf + 1;   // [2] a round of the bank is complete (round schedule)
-  uint64_t* bankfree = bankfull + 2;  // [2] the bank has been added into registers
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bankfree + 2);
+  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + S * SM::kStage);
+  uint64_t* conv = full + S;
+  uint64_t* empty = conv + S;
+  uint64_t* accf = empty + S;
+  uint64_t* bfull = accf + 1;  // [2] a round of the bank is complete (round schedule)
+  uint64_t* bfree = bfull + 2; // [2] the bank has been added into registers
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bfree + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -119,19 +104,15 @@ __global__ void __launch_bounds__(192, 1)
   const int nk = (K + kBK - 1) / kBK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SR; ++s) {
-      mbar_init(&rawfull[s], 1);
-      mbar_init(&rawfree[s], 128);
-    }
-    for (int s = 0; s < SO; ++s) {
-      mbar_init(&opfull[s], 1);
-      mbar_init(&opconv[s], 128);
-      mbar_init(&opfree[s], 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&conv[s], 128);
+      mbar_init(&empty[s], 1);
     }
     mbar_init(accf, 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&bankfull[b], 1);
-      mbar_init(&bankfree[b], 128);
+      mbar_init(&bfull[b], 1);
+      mbar_init(&bfree[b], 128);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -142,53 +123,42 @@ __global__ void __launch_bounds__(192, 1)
   fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  auto sRaw = [&](int r) { return raw_base + r * SM::kA; };
-  auto sA = [&](int c) { return op_base + c * SM::kOpStage; };
-  auto sAlo = [&](int c) { return op_base + c * SM::kOpStage + SM::kA; };
-  auto sB = [&](int c) { return op_base + c * SM::kOpStage + (SPLIT ? 2 : 1) * SM::kA; };
-  auto sBlo = [&](int c) { return op_base + c * SM::kOpStage + 2 * SM::kA + SM::kB; };
+  auto sA = [&](int s) { return base + s * SM::kStage; };
+  auto sAlo = [&](int s) { return base + s * SM::kStage + SM::kA; };
+  auto sB = [&](int s) { return base + s * SM::kStage + 2 * SM::kA; };
+  auto sBlo = [&](int s) { return base + s * SM::kStage + 2 * SM::kA + SM::kB; };
 
-  int issued = 0;  // K steps whose loads this producer lane issued
-  if (warp == 0 && lane < (SPLIT ? 2 : 1)) {
-    // lane 0: A tiles (3xTF32: into the raw ring); lane 1 (3xTF32): the B halves into the operand stages
-    const bool a_lane = lane == 0;
-    for (int kt = 0; kt < nk; ++kt) {
-      const bool into_raw = SPLIT && a_lane;
-      const int S = into_raw ? SR : SO, s = kt % S;
-      uint64_t* freeb = into_raw ? &rawfree[s] : &opfree[s];
-      if (kt >= S && !mbar_wait(freeb, ((kt / S) + 1) & 1, limit, 1)) {
-        *abort_flag = 1;
-        break;
+  int issued = 0;  // TMA stages issued by warp 0
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t bytes = SM::kA + (SPLIT ? 2 : 1) * SM::kB;
+      for (int kt = 0; kt < nk; ++kt) {
+        const int s = kt % S;
+        if (kt >= S && !mbar_wait(&empty[s], ((kt / S) + 1) & 1, limit, 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        if (*abort_flag) break;
+        mbar_expect_tx(&full[s], bytes);
+        tma_load_2d(sA(s), &tmA, &full[s], kt * kBK, m0);
+        tma_load_2d(sB(s), &tmB, &full[s], kt * kBK, n0);
+        if (SPLIT) tma_load_2d(sBlo(s), &tmBlo, &full[s], kt * kBK, n0);
+        issued = kt + 1;
       }
-      if (*abort_flag) break;
-      if (into_raw) {
-        mbar_expect_tx(&rawfull[s], SM::kA);
-        tma_load_2d(sRaw(s), &tmA, &rawfull[s], kt * kBK, m0);
-      } else if (SPLIT) {
-        mbar_expect_tx(&opfull[s], 2 * SM::kB);
-        tma_load_2d(sB(s), &tmB, &opfull[s], kt * kBK, n0);
-        tma_load_2d(sBlo(s), &tmBlo, &opfull[s], kt * kBK, n0);
-      } else {
-        mbar_expect_tx(&opfull[s], SM::kA + SM::kB);
-        tma_load_2d(sA(s), &tmA, &opfull[s], kt * kBK, m0);
-        tma_load_2d(sB(s), &tmB, &opfull[s], kt * kBK, n0);
-      }
-      issued = kt + 1;
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_tf32(kBM, BN);
       for (int kt = 0; kt < nk; ++kt) {
-        const int s = kt % SO;
-        const uint32_t par = (kt / SO) & 1;
+        const int s = kt % S;
+        const uint32_t par = (kt / S) & 1;
         // round schedule: round r = kt / D writes bank r & 1, free again once round r - 2 was drained
         const int r = DRAIN ? kt / RS::D : 0, j = DRAIN ? kt - r * RS::D : kt, bank = r & 1;
-        if (DRAIN && j == 0 && r >= 2 && !mbar_wait(&bankfree[bank], ((r >> 1) - 1) & 1, limit, 7)) {
+        if (DRAIN && j == 0 && r >= 2 && !mbar_wait(&bfree[bank], ((r >> 1) - 1) & 1, limit, 7)) {
           *abort_flag = 1;
           break;
         }
-        if (!mbar_wait(&opfull[s], par, limit, 2) || (SPLIT && !mbar_wait(&opconv[s], par, limit, 2)) ||
-            *abort_flag) {
+        if (!mbar_wait(SPLIT ? &conv[s] : &full[s], par, limit, 2) || *abort_flag) {
           *abort_flag = 1;
           break;
         }
@@ -207,15 +177,14 @@ __global__ void __launch_bounds__(192, 1)
             mma_tf32(td, sw128_kmajor(al + off), sw128_kmajor(b + off), idesc, 1u);
           }
         }
-        mma_commit(&opfree[s]);
-        if (DRAIN && (j == RS::D - 1 || kt == nk - 1)) mma_commit(&bankfull[bank]);
+        mma_commit(&empty[s]);
+        if (DRAIN && (j == RS::D - 1 || kt == nk - 1)) mma_commit(&bfull[bank]);
       }
       mma_commit(accf);
     }
-  } else if (warp >= 2) {
-    // warps 2..5: split A into the operand stages (3xTF32), add finished rounds
-    // of accumulators into registers, then the epilogue.  Every exit decision of
-    // these warps is warp-uniform (__all_sync): the TMEM loads are warp-collective.
+  } else {
+    // warps 2..5: split A in shared memory (3xTF32), add finished rounds of
+    // accumulators into registers, then the epilogue
     const int t = threadIdx.x - 64;  // 0..127
     const int q = warp & 3;          // TMEM lane quadrant this warp may access
     const uint32_t tlane = tmem + (uint32_t(q * 32) << 16);
@@ -224,37 +193,30 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
     for (int i = 0; i < NR; ++i) racc[i] = 0.f;
     int drained = 0;  // rounds added into racc
+    // every exit decision of these warps is made warp-uniform (__all_sync): the
+    // TMEM loads below are warp-collective
     auto drain = [&](int rr) -> bool {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bankfull[rr & 1], (rr >> 1) & 1, limit, 8))) return false;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bfull[rr & 1], (rr >> 1) & 1, limit, 8))) return false;
       fence_after_sync();
       tmem_drain<NR, RS::NPB>(tlane, rr & 1, min(RS::NPB, RS::steps(rr, nk)), kCols, racc);
       fence_before_sync();
-      mbar_arrive(&bankfree[rr & 1]);
+      mbar_arrive(&bfree[rr & 1]);
       ++drained;
       return true;
     };
-    if constexpr (SPLIT) {
+    if (SPLIT) {
       for (int kt = 0; kt < nk; ++kt) {
-        const int r = kt % SR, s = kt % SO;
-        const bool got = mbar_wait(&rawfull[r], (kt / SR) & 1, limit, 3) &&
-                         (kt < SO || mbar_wait(&opfree[s], ((kt / SO) + 1) & 1, limit, 3)) && !*abort_flag;
-        if (!__all_sync(0xffffffffu, got)) {
+        const int s = kt % S;
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (kt / S) & 1, limit, 3) && !*abort_flag)) {
           *abort_flag = 1;
           break;
         }
-        const float4* r4 = reinterpret_cast<const float4*>(sRaw(r));
-        float4* h4 = reinterpret_cast<float4*>(sA(s));
+        float4* a4 = reinterpret_cast<float4*>(sA(s));
         float4* l4 = reinterpret_cast<float4*>(sAlo(s));
 #pragma unroll 4
-        for (int i = t; i < kBM * kBK / 4; i += 128) {
-          float4 v = r4[i];
-          h4[i] = v;
-          split4(h4 + i, l4 + i);
-        }
-        // the MMA (async proxy) reads the halves; TMA may refill the raw tile
+        for (int i = t; i < kBM * kBK / 4; i += 128) split4(a4 + i, l4 + i);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive(&opconv[s]);
-        mbar_arrive(&rawfree[r]);
+        mbar_arrive(&conv[s]);
         if constexpr (DRAIN) {
           const int rr = RS::drain_after(kt);
           if (rr >= 0 && !drain(rr)) {
@@ -295,15 +257,15 @@ __global__ void __launch_bounds__(192, 1)
             float4* d4 = reinterpret_cast<float4*>(dst0);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              float4 t4 = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+              float4 t = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
               if (accumulate) {
                 const float4 o = d4[i];
-                t4.x += o.x;
-                t4.y += o.y;
-                t4.z += o.z;
-                t4.w += o.w;
+                t.x += o.x;
+                t.y += o.y;
+                t.z += o.z;
+                t.w += o.w;
               }
-              d4[i] = t4;
+              d4[i] = t;
             }
           } else {
 #pragma unroll
@@ -319,14 +281,13 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   }
-  // before exit: every copy a producer lane issued has landed (bounded wait),
-  // and the MMA thread's own MMAs have completed; then TMEM is released
-  if (warp == 0 && lane < (SPLIT ? 2 : 1) && *abort_flag) {
-    const bool into_raw = SPLIT && lane == 0;
-    const int S = into_raw ? SR : SO;
+  // drain: the producer waits (bounded) for the loads it issued so no copy is
+  // in flight when the CTA exits, then TMEM is released
+  if (warp == 0 && lane == 0 && *abort_flag) {
     for (int kt = (issued > S ? issued - S : 0); kt < issued; ++kt)
-      mbar_wait(into_raw ? &rawfull[kt % S] : &opfull[kt % S], (kt / S) & 1, kDrainLimitNs, 5);
+      mbar_wait(&full[kt % S], (kt / S) & 1, kDrainLimitNs, 5);
   }
+  // the MMA thread waits for its own MMAs before TMEM is released
   if (warp == 1 && lane == 0) mbar_wait(accf, 0, kDrainLimitNs, 6);
   fence_before_sync();
   __syncthreads();
@@ -375,7 +336,7 @@ cudaError_t run(const float* A, int64_t lda, const float* B, const float* Blo, i
   if (!make_map(&ta, A, M, K, lda, kBM) || !make_map(&tb, B, N, K, ldb, BN)) return cudaErrorInvalidValue;
   if (SPLIT && !make_map(&tbl, Blo, N, K, ldb, BN)) return cudaErrorInvalidValue;
   if (!SPLIT) tbl = tb;
-  using SM = TcSmem<BN, SPLIT>;
+  using SM = TcSmem<BN>;
   dim3 grid(unsigned((M + kBM - 1) / kBM), unsigned((N + BN - 1) / BN));
   k_gemm_tc<BN, SPLIT><<<grid, 192, SM::kBytes, st>>>(ta, tb, tbl, M, N, K, out, accumulate, limit);
   return cudaGetLastError();
@@ -383,8 +344,7 @@ cudaError_t run(const float* A, int64_t lda, const float* B, const float* Blo, i
 
 template <int BN, bool SPLIT>
 cudaError_t set_smem() {
-  return cudaFuncSetAttribute(k_gemm_tc<BN, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              TcSmem<BN, SPLIT>::kBytes);
+  return cudaFuncSetAttribute(k_gemm_tc<BN, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcSmem<BN>::kBytes);
 }
 
 }  // namespace
