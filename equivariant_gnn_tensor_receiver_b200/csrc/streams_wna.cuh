@@ -1,11 +1,13 @@
 // Warp-per-node receiver adjoint streams, lane = edge (first and second order).
 //
-// One warp owns one receiver r and walks its CSR segment in batches of 32
-// edges, one edge per lane.  The node-side adjoint state G = Theta^T g_r (and,
-// for the double backward, Gt = gg_Theta^T g_r) is staged by cp.async in chunks
-// of kWnChunk channels as [u][k][m3], so that every lane reads a channel's
-// RM x n3 block with broadcast 16-byte loads, while each lane stages and reads
-// its own edge's sender row.  All reductions over channels happen in the lane's
+// A warp takes 32 consecutive edges of the receiver-sorted CSR order (one per
+// lane), whichever receivers they belong to: every lane does useful work, and a
+// hub's edges spread over many warps.  The node-side adjoint state
+// G = Theta^T g_r (and, for the double backward, Gt = gg_Theta^T g_r) of the
+// receivers present is staged by cp.async in chunks of kWnChunk channels as
+// [u][k][m3], one slot per receiver, so that the lanes of one receiver read a
+// channel's RM x n3 block with broadcast 16-byte loads, while each lane stages
+// and reads its own edge's sender row.  All reductions over channels happen in the lane's
 // registers; the CG contraction with the per-edge outer-product accumulator Q
 // runs once per path rather than once per channel.
 //
@@ -97,9 +99,13 @@ __host__ __device__ constexpr int g_slot(int k, int m3) {
 }
 
 // one path of one 32-edge batch (GT: the second order has a Gt operand)
+// rfirst: chunk-local receiver of lane 0's edge; the window's receivers are
+// rfirst .. rfirst + nslots - 1 and the lane's is rfirst + myslot (myslot < 0:
+// no edge).
 template <int L1, int L2, int L3, int RM, bool DBL, bool GT>
-__device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, const WnaLay& L, float* ws, int rl,
-                                         int nc, int nb, int myrow, const float* __restrict__ x,
+__device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, const WnaLay& L, float* ws, int rfirst,
+                                         int nslots, int myslot, int nc, int nb, int myrow,
+                                         const float* __restrict__ x,
                                          const float* __restrict__ x1, const float* __restrict__ G,
                                          const float* __restrict__ Gt, float2* db, float2* hb) {
   using TR = Tri<L1, L2, L3>;
@@ -145,9 +151,11 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
   const int Kb = pl.Kb[q.i3];
   constexpr bool has_t = DBL && GT;
   const bool has_x1 = DBL && x1 != nullptr;
-  // this lane's G elements of a chunk: source offset (relative to channel u0)
-  // and shared slot, the same for every chunk of the path
-  const float* Gp = G + size_t(nc) * pl.a_pref[q.i3] + size_t(rl) * N3 * Kb + q.koff;
+  // this lane's G elements of a chunk: source offset (relative to receiver row
+  // and channel u0) and position inside a slot, the same for every chunk
+  constexpr int NS = kWnaSlots(DBL);
+  const size_t rowstride = size_t(N3) * Kb;
+  const float* Gp = G + size_t(nc) * pl.a_pref[q.i3] + size_t(rfirst) * rowstride + q.koff;
   const float* Gtp = has_t ? Gt + (Gp - G) : nullptr;
   int gsrc[NIT], gdst[NIT];
 #pragma unroll
@@ -158,15 +166,20 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
     gsrc[it] = k < R ? m3 * Kb + k * c + u : -1;
     gdst[it] = u * GW + g_slot<N3>(k, m3);
   }
+  int g0 = 0;  // first receiver slot of the group being staged
   auto stage = [&](int ch) {
     const int u0 = ch * CH;
-    float* sG = ws + L.G + (ch & 1) * L.gbuf;
-    float* sGt = ws + L.Gt + (ch & 1) * L.gbuf;
+    const int ns = min(NS, nslots - g0);
+    for (int sl = 0; sl < ns; ++sl) {
+      float* sG = ws + L.G + (ch & 1) * L.gbuf + sl * L.gslot;
+      float* sGt = ws + L.Gt + (ch & 1) * L.gbuf + sl * L.gslot;
+      const size_t ro = size_t(g0 + sl) * rowstride + u0;
 #pragma unroll
-    for (int it = 0; it < NIT; ++it) {
-      if (gsrc[it] >= 0) {
-        ac_copy4(sG + gdst[it], Gp + u0 + gsrc[it]);
-        if constexpr (has_t) ac_copy4(sGt + gdst[it], Gtp + u0 + gsrc[it]);
+      for (int it = 0; it < NIT; ++it) {
+        if (gsrc[it] >= 0) {
+          ac_copy4(sG + gdst[it], Gp + ro + gsrc[it]);
+          if constexpr (has_t) ac_copy4(sGt + gdst[it], Gtp + ro + gsrc[it]);
+        }
       }
     }
     // the batch's rows, N1 16-byte pieces each, copied by the whole warp (coalesced)
@@ -186,6 +199,11 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
     }
   };
 
+  // receivers in groups of NS slots (one group unless the window spans more
+  // than NS receivers); a lane whose receiver is not in the group reads the
+  // zero slot, which adds nothing to its sums
+  for (g0 = 0; g0 < nslots; g0 += NS) {
+  const bool active = myslot >= g0 && myslot < g0 + NS;
   if (nch > 0) stage(0);
   ac_commit();
   for (int ch = 0; ch < nch; ++ch) {
@@ -193,8 +211,8 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
     ac_commit();
     ac_wait<1>();
     __syncwarp();
-    const float* sG = ws + L.G + (ch & 1) * L.gbuf;
-    const float* sGt = ws + L.Gt + (ch & 1) * L.gbuf;
+    const float* sG = active ? ws + L.G + (ch & 1) * L.gbuf + (myslot - g0) * L.gslot : ws + L.Z;
+    const float* sGt = active ? ws + L.Gt + (ch & 1) * L.gbuf + (myslot - g0) * L.gslot : ws + L.Z;
     // the lane's four channels in N1 16-byte reads
     float xg[CH * N1], x1g[DBL ? CH * N1 : 1];
     lds_vec<CH * N1>(ws + L.X + (ch & 1) * L.xbuf + lane * L.xs, xg);
@@ -274,6 +292,7 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
     }
     __syncwarp();
   }
+  }  // receiver groups
   // this path's share of dY (second order: wY, hY) for the lane's edge
   float* acc = ws + L.Acc + lane * L.accs;
   float o[N2];
@@ -292,15 +311,15 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
 }
 
 // Persistent grid of kWnWarps-warp CTAs.  A CTA takes kWnWarps work items per
-// round from *counter; an item is one batch of up to 32 edges of a receiver:
-// item t < nc is receiver t's first batch, item t >= nc a further batch (list
-// `extra`, built with seg = 32).  The warps of a CTA step through the paths
-// together (one barrier per path), so the resident warps of an SM share one or
-// two path bodies in the instruction caches, and every warp of a round has at
-// most one batch, so the rounds stay balanced whatever the degrees.
+// round from *counter; an item is a window of 32 consecutive edges of the
+// chunk's receiver-sorted CSR range (one edge per lane), whichever receivers
+// they belong to, so every lane but those of the range's last window has an
+// edge.  The warps of a CTA step through the paths together (one barrier per
+// path), so the resident warps of an SM share one or two path bodies in the
+// instruction caches, and the rounds stay balanced whatever the degrees.
 // First order writes dvec (and, when given, dY [E][n_sh], db [E][R]); second
 // order writes dvec.  x1 / ggv may be null (their terms vanish); Gt is used
-// exactly when GT.
+// exactly when GT.  The counter is reset by the caller before the launch.
 template <int RM, int LF, bool DBL, bool GT>
 __global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
     k_wn_adj(const __grid_constant__ DevPlan pl, int r0, int nc, const int* __restrict__ rowptr,
@@ -313,9 +332,11 @@ __global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
   const WnaLay L = wna_layout_of(RM, pl.n3max, pl.n1max, DBL);
   float* ws = sm + warp * L.total;
   int& s_base = *reinterpret_cast<int*>(sm + kWnWarps * L.total);  // this round's first item
-  // staged buffers read where nothing was staged must hold zeros
+  (void)extra;
+  // staged buffers read where nothing was staged (and the zero slot) must hold zeros
   for (int i = lane; i < L.Geo; i += 32) ws[i] = 0.f;
-  const int total = nc + extra[nc];
+  const int e_lo = rowptr[r0], e_hi = rowptr[r0 + nc];
+  const int total = (e_hi - e_lo + kBatchEdges - 1) / kBatchEdges;
   // the next round is claimed while the current one runs (hides the atomic's latency)
   int claim = threadIdx.x == 0 ? atomicAdd(counter, kWnWarps) : 0;
   for (;;) {
@@ -327,20 +348,28 @@ __global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
     __syncthreads();
     const int t = s_base + warp;
     if (s_base >= total) break;  // uniform over the CTA
-    int rl = -1, eb = 0, nb = 0;
+    int eb = 0, nb = 0;
     if (t < total) {
-      rl = t;
-      int k = 0;
-      if (t >= nc) {
-        rl = extra_owner(extra, nc, t - nc);
-        k = 1 + (t - nc - extra[rl]);
-      }
-      const int e0 = rowptr[r0 + rl], e1 = rowptr[r0 + rl + 1];
-      eb = e0 + kBatchEdges * k;
-      nb = max(0, min(kBatchEdges, e1 - eb));
+      eb = e_lo + kBatchEdges * t;
+      nb = min(kBatchEdges, e_hi - eb);
     }
     const bool valid = lane < nb;
     const int e = eb + lane;
+    // the lane's receiver (chunk-local): the last node whose segment starts at or before e
+    int rl = 0;
+    if (valid) {
+      int lo = 0, hi = nc;  // rowptr[r0 + lo] <= e < rowptr[r0 + hi]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (rowptr[r0 + mid] <= e) lo = mid;
+        else hi = mid;
+      }
+      rl = lo;
+    }
+    const int rfirst = __shfl_sync(0xffffffffu, rl, 0);
+    const int rlast = __shfl_sync(0xffffffffu, rl, nb > 0 ? nb - 1 : 0);
+    const int nslots = nb > 0 ? rlast - rfirst + 1 : 0;
+    const int myslot = valid ? rl - rfirst : -1;
     int myrow = 0;
     float* geo = ws + L.Geo + lane * L.geos;
     float* acc = ws + L.Acc + lane * L.accs;
@@ -388,7 +417,8 @@ __global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
 #define TPC_CASE(a, b, c)                                                                                 \
   case triple_id(a, b, c):                                                                                \
     if constexpr (a <= LF && c <= LF)                                                                     \
-      wna_path<a, b, c, RM, DBL, GT>(pl, q, L, ws, rl, nc, nb, myrow, x, x1, G, Gt, db2, hb2);              \
+      wna_path<a, b, c, RM, DBL, GT>(pl, q, L, ws, rfirst, nslots, myslot, nc, nb, myrow, x, x1, G, Gt, db2, \
+                                     hb2);                                                                \
     break;
           TPC_FOR_EACH_TRIPLE(TPC_CASE)
 #undef TPC_CASE

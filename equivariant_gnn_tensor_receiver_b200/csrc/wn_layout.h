@@ -47,23 +47,31 @@ TPC_HD inline int wn_smem_bytes(int RM, int cpl, int nimax, int nmz_max, bool db
 }
 
 // ---- lane = edge (receiver adjoint streams, first and second order) --------
-// G, Gt : two chunk buffers of kWnChunk channels of G (and Gt), [u][k/2][m3][k&1]
-//         with row stride RM * (2 l3 + 1) of the path (zero where never staged)
+// A warp's lanes are 32 consecutive CSR edges, which may belong to several
+// receivers; the G rows of up to kWnaSlots(dbl) of them are staged at once.
+// G, Gt : two chunk buffers, each kWnaSlots slots of kWnChunk channels of one
+//         receiver's G (and Gt), [u][k/2][m3][k&1] with row stride
+//         RM * (2 l3 + 1) of the path (zero where never staged); slot stride
+//         gslot = kWnChunk * gs + 4 floats, so that lanes reading different
+//         slots fall into different bank quads
+// Z     : one slot of zeros, read by lanes whose receiver is not staged
 // X, X1 : two chunk buffers of the 32 lanes' rows, [lane][u * n1 + m1] with row
 //         stride xs, xs / 4 odd: the 16-byte reads of 8 consecutive lanes fall
 //         into distinct bank quads
 // Geo   : per lane Y[16], b[RM] (and Yd[16], bd[RM]), odd stride
 // Acc   : per lane accumulators that persist across paths (dY, or wY and hY), odd stride
+TPC_HD constexpr int kWnaSlots(bool dbl) { return dbl ? 2 : 4; }
 struct WnaLay {
-  int G, Gt, X, X1, Geo, Acc;
-  int gs, gbuf, xs, xbuf, geos, accs;
+  int G, Gt, Z, X, X1, Geo, Acc;
+  int gs, gslot, gbuf, xs, xbuf, geos, accs;
   int total;
 };
 
 TPC_HD inline WnaLay wna_layout_of(int RM, int n3max, int n1max, bool dbl) {
   WnaLay L;
   L.gs = RM * n3max;
-  L.gbuf = kWnChunk * L.gs;
+  L.gslot = kWnChunk * L.gs + 4;
+  L.gbuf = kWnaSlots(dbl) * L.gslot;
   L.xs = (kWnChunk * n1max + 3) & ~3;
   if ((L.xs >> 2) % 2 == 0) L.xs += 4;
   L.xbuf = 32 * L.xs;
@@ -71,7 +79,8 @@ TPC_HD inline WnaLay wna_layout_of(int RM, int n3max, int n1max, bool dbl) {
   L.accs = (dbl ? 32 : 16) + 1;
   L.G = 0;
   L.Gt = L.G + 2 * L.gbuf;
-  L.X = L.Gt + (dbl ? 2 * L.gbuf : 0);
+  L.Z = L.Gt + (dbl ? 2 * L.gbuf : 0);
+  L.X = L.Z + L.gslot;
   L.X1 = L.X + 2 * L.xbuf;
   L.Geo = L.X1 + (dbl ? 2 * L.xbuf : 0);
   L.Acc = L.Geo + 32 * L.geos;
@@ -85,7 +94,7 @@ TPC_HD inline int wna_smem_bytes(int RM, int n3max, int n1max, bool dbl) {
 
 // ---- work items of the streams (lists built in graph.cuh) ----
 // Item t < nc is node t's first piece; item t >= nc is extra piece t - nc.
-constexpr int kBatchEdges = 32;  // edges per adjoint work item (lane = edge)
+constexpr int kBatchEdges = 32;  // edges per adjoint work item (lane = edge): 32 consecutive CSR edges
 
 #if defined(__CUDACC__)
 // item t >= nc: the extra piece u = t - nc belongs to the node i with extra[i] <= u < extra[i+1]
