@@ -1,5 +1,5 @@
 // Host-side launchers of the edge-stream kernels.  Each kernel family is
-// instantiated per radial register width RM (4, 8, 16) in its own translation
+// instantiated per radial register width RM (8, 16) in its own translation
 // unit (tu_*.cu); every unit registers an initialiser that uploads its copy of
 // the constant CG table and raises its kernels' shared-memory limit.
 #pragma once
@@ -60,17 +60,13 @@ cudaError_t launch_wn_dadj(const DevPlan& d, int r0, int nc, const int* rowptr, 
                            float* dvec, const int* extra, int* counter, cudaStream_t st);
 
 // instantiation of a warp-per-node launcher for the plan's (rm, wn_lf[, wn_cpl])
-#define TPC_WN_CALL(d, fn, ...)                                                                \
-  ((d).rm == 4 ? fn<4, 3>(__VA_ARGS__)                                                         \
-               : (d).rm == 16 ? fn<16, 3>(__VA_ARGS__)                                         \
-                              : (d).wn_lf == 2 ? fn<8, 2>(__VA_ARGS__) : fn<8, 3>(__VA_ARGS__))
+#define TPC_WN_CALL(d, fn, ...) \
+  ((d).rm == 16 ? fn<16, 3>(__VA_ARGS__) : (d).wn_lf == 2 ? fn<8, 2>(__VA_ARGS__) : fn<8, 3>(__VA_ARGS__))
 #define TPC_WN_CALL_CPL(d, fn, ...)                                                                     \
-  ((d).rm == 4    ? fn<4, 3, 1>(__VA_ARGS__)                                                            \
-   : (d).rm == 16 ? fn<16, 3, 1>(__VA_ARGS__)                                                           \
+  ((d).rm == 16      ? fn<16, 3, 1>(__VA_ARGS__)                                                        \
    : (d).wn_lf == 2 ? ((d).wn_cpl == 2 ? fn<8, 2, 2>(__VA_ARGS__) : fn<8, 2, 1>(__VA_ARGS__))           \
                     : fn<8, 3, 1>(__VA_ARGS__))
 
-#define TPC_RM_CALL(rm, fn, ...) \
-  ((rm) == 4 ? fn<4>(__VA_ARGS__) : (rm) == 8 ? fn<8>(__VA_ARGS__) : fn<16>(__VA_ARGS__))
+#define TPC_RM_CALL(rm, fn, ...) ((rm) == 8 ? fn<8>(__VA_ARGS__) : fn<16>(__VA_ARGS__))
 
 }  // namespace tpc

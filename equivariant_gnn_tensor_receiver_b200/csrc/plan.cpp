@@ -343,7 +343,7 @@ int tpconv_plan_create(tpconv_plan** out, const char* irreps_in, int l_sh_max,
       }
   d.P = P;
   d.family = o.family;
-  d.rm = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
+  d.rm = R <= 8 ? 8 : 16;  // radial registers per lane; entries k >= R stay zero
   int sm = 0, sm2 = 0;
   for (int i = 0; i < P; ++i) {
     DevPath& q = d.path[i];

@@ -108,7 +108,7 @@ struct DevPlan {
   int Kx[kMaxBlocks];               // columns of the B block of input block i1
   int64_t b_pref[kMaxBlocks + 1];   // floats per node before block i1 (sum n1 * Kx)
   int max_c_in, max_c_out;
-  int rm;                           // radial registers per lane (4, 8 or 16) >= R
+  int rm;                           // radial registers per lane (8 or 16) >= R
   int sm_floats;                    // dynamic smem floats of the per-path adjoint stream
   int sm_floats2;                   // the same for its double-backward form
   int wn_ok;                        // rows stageable 16 bytes at a time (channel counts multiple of 4)
