@@ -1,8 +1,10 @@
 // Warp-per-node receiver adjoint streams, lane = edge (first and second order).
 //
-// A warp takes 32 consecutive edges of the receiver-sorted CSR order (one per
-// lane), whichever receivers they belong to: every lane does useful work, and a
-// hub's edges spread over many warps.  The node-side adjoint state
+// Second order: a warp takes 32 consecutive edges of the receiver-sorted CSR
+// order (one per lane), whichever receivers they belong to, so every lane does
+// useful work; first order (lighter per channel, where staging several
+// receivers' rows costs more than the idle lanes): up to 32 edges of one
+// receiver.  Either way a hub's edges spread over many warps.  The node-side adjoint state
 // G = Theta^T g_r (and, for the double backward, Gt = gg_Theta^T g_r) of the
 // receivers present is staged by cp.async in chunks of kWnChunk channels as
 // [u][k][m3], one slot per receiver, so that the lanes of one receiver read a
@@ -311,12 +313,14 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
 }
 
 // Persistent grid of kWnWarps-warp CTAs.  A CTA takes kWnWarps work items per
-// round from *counter; an item is a window of 32 consecutive edges of the
-// chunk's receiver-sorted CSR range (one edge per lane), whichever receivers
-// they belong to, so every lane but those of the range's last window has an
-// edge.  The warps of a CTA step through the paths together (one barrier per
-// path), so the resident warps of an SM share one or two path bodies in the
-// instruction caches, and the rounds stay balanced whatever the degrees.
+// round from *counter.  Second order: an item is a window of 32 consecutive
+// edges of the chunk's receiver-sorted CSR range (one edge per lane), whichever
+// receivers they belong to.  First order: an item is one batch of up to 32
+// edges of a receiver: item t < nc is receiver t's first batch, item t >= nc a
+// further batch (list `extra`, built with seg = 32).  The warps of a CTA step
+// through the paths together (one barrier per path), so the resident warps of
+// an SM share one or two path bodies in the instruction caches, and the rounds
+// stay balanced whatever the degrees.
 // First order writes dvec (and, when given, dY [E][n_sh], db [E][R]); second
 // order writes dvec.  x1 / ggv may be null (their terms vanish); Gt is used
 // exactly when GT.  The counter is reset by the caller before the launch.
@@ -332,11 +336,10 @@ __global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
   const WnaLay L = wna_layout_of(RM, pl.n3max, pl.n1max, DBL);
   float* ws = sm + warp * L.total;
   int& s_base = *reinterpret_cast<int*>(sm + kWnWarps * L.total);  // this round's first item
-  (void)extra;
   // staged buffers read where nothing was staged (and the zero slot) must hold zeros
   for (int i = lane; i < L.Geo; i += 32) ws[i] = 0.f;
   const int e_lo = rowptr[r0], e_hi = rowptr[r0 + nc];
-  const int total = (e_hi - e_lo + kBatchEdges - 1) / kBatchEdges;
+  const int total = DBL ? (e_hi - e_lo + kBatchEdges - 1) / kBatchEdges : nc + extra[nc];
   // the next round is claimed while the current one runs (hides the atomic's latency)
   int claim = threadIdx.x == 0 ? atomicAdd(counter, kWnWarps) : 0;
   for (;;) {
@@ -348,28 +351,42 @@ __global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
     __syncthreads();
     const int t = s_base + warp;
     if (s_base >= total) break;  // uniform over the CTA
-    int eb = 0, nb = 0;
-    if (t < total) {
-      eb = e_lo + kBatchEdges * t;
-      nb = min(kBatchEdges, e_hi - eb);
+    int eb = 0, nb = 0, rfirst = 0, nslots = 0, myslot = -1;
+    if constexpr (DBL) {
+      if (t < total) {
+        eb = e_lo + kBatchEdges * t;
+        nb = min(kBatchEdges, e_hi - eb);
+      }
+      // the lane's receiver (chunk-local): the last node whose segment starts at or before its edge
+      int rl = 0;
+      if (lane < nb) {
+        int lo = 0, hi = nc;  // rowptr[r0 + lo] <= e < rowptr[r0 + hi]
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (rowptr[r0 + mid] <= eb + lane) lo = mid;
+          else hi = mid;
+        }
+        rl = lo;
+      }
+      rfirst = __shfl_sync(0xffffffffu, rl, 0);
+      const int rlast = __shfl_sync(0xffffffffu, rl, nb > 0 ? nb - 1 : 0);
+      nslots = nb > 0 ? rlast - rfirst + 1 : 0;
+      myslot = lane < nb ? rl - rfirst : -1;
+    } else if (t < total) {
+      int rl = t, k = 0;
+      if (t >= nc) {
+        rl = extra_owner(extra, nc, t - nc);
+        k = 1 + (t - nc - extra[rl]);
+      }
+      const int e0 = rowptr[r0 + rl], e1 = rowptr[r0 + rl + 1];
+      eb = e0 + kBatchEdges * k;
+      nb = max(0, min(kBatchEdges, e1 - eb));
+      rfirst = rl;
+      nslots = nb > 0 ? 1 : 0;
+      myslot = lane < nb ? 0 : -1;
     }
     const bool valid = lane < nb;
     const int e = eb + lane;
-    // the lane's receiver (chunk-local): the last node whose segment starts at or before e
-    int rl = 0;
-    if (valid) {
-      int lo = 0, hi = nc;  // rowptr[r0 + lo] <= e < rowptr[r0 + hi]
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (rowptr[r0 + mid] <= e) lo = mid;
-        else hi = mid;
-      }
-      rl = lo;
-    }
-    const int rfirst = __shfl_sync(0xffffffffu, rl, 0);
-    const int rlast = __shfl_sync(0xffffffffu, rl, nb > 0 ? nb - 1 : 0);
-    const int nslots = nb > 0 ? rlast - rfirst + 1 : 0;
-    const int myslot = valid ? rl - rfirst : -1;
     int myrow = 0;
     float* geo = ws + L.Geo + lane * L.geos;
     float* acc = ws + L.Acc + lane * L.accs;

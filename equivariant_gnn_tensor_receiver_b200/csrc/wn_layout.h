@@ -47,8 +47,10 @@ TPC_HD inline int wn_smem_bytes(int RM, int cpl, int nimax, int nmz_max, bool db
 }
 
 // ---- lane = edge (receiver adjoint streams, first and second order) --------
-// A warp's lanes are 32 consecutive CSR edges, which may belong to several
-// receivers; the G rows of up to kWnaSlots(dbl) of them are staged at once.
+// Second order: a warp's lanes are 32 consecutive CSR edges, which may belong
+// to several receivers; the G rows of up to kWnaSlots(true) of them are staged
+// at once.  First order: a warp's lanes are up to 32 edges of one receiver
+// (one slot).
 // G, Gt : two chunk buffers, each kWnaSlots slots of kWnChunk channels of one
 //         receiver's G (and Gt), [u][k/2][m3][k&1] with row stride
 //         RM * (2 l3 + 1) of the path (zero where never staged); slot stride
@@ -60,7 +62,7 @@ TPC_HD inline int wn_smem_bytes(int RM, int cpl, int nimax, int nmz_max, bool db
 //         into distinct bank quads
 // Geo   : per lane Y[16], b[RM] (and Yd[16], bd[RM]), odd stride
 // Acc   : per lane accumulators that persist across paths (dY, or wY and hY), odd stride
-TPC_HD constexpr int kWnaSlots(bool dbl) { return dbl ? 2 : 4; }
+TPC_HD constexpr int kWnaSlots(bool dbl) { return dbl ? 2 : 1; }
 struct WnaLay {
   int G, Gt, Z, X, X1, Geo, Acc;
   int gs, gslot, gbuf, xs, xbuf, geos, accs;
