@@ -359,10 +359,19 @@ def parity_check(args, work, graph, procs, k):
     import torch
     rowptr, col, vec = graph
     N, E = work.N, work.E
+    # host inputs stay fp32 views of the pinned buffers; only the rows a job
+    # needs are widened to fp64, and only sampled rows of the outputs come back
+    # from the device (the capacity workload's full arrays are tens of GB)
     h = {key: v.numpy() for key, v in work.host.items()}
-    f64 = lambda a: np.asarray(a, dtype=np.float32).astype(np.float64)
-    x, th, g, ggx, ggv, v32 = (f64(h[key]) for key in ("x", "theta", "g", "gg_x", "gg_vec", "vec"))
-    gpu = {key: t.double().cpu().numpy() for key, t in work.outs.items()}
+    x, g, ggx, ggv, v32 = (h[key] for key in ("x", "g", "gg_x", "gg_vec", "vec"))
+    th = h["theta"].astype(np.float64)
+    f64 = lambda a: np.asarray(a, dtype=np.float64)
+
+    def gpu_rows(key, idx):
+        t = work.outs[key]
+        return t.index_select(0, torch.as_tensor(idx, dtype=torch.int64, device=t.device)).double().cpu().numpy()
+
+    gpu = {key: work.outs[key].double().cpu().numpy() for key in ("dtheta", "d_theta")}
     rng = np.random.default_rng(12345)
     recv_all = np.repeat(np.arange(N), np.diff(np.asarray(rowptr, dtype=np.int64)))
     k_dbl = max(1, k // 4)
@@ -374,8 +383,8 @@ def parity_check(args, work, graph, procs, k):
 
     def job(kind, edges):
         lrp, lc, eids, recvs, nodes = _sub_problem(rowptr, col, edges)
-        a = {"rowptr": lrp, "col": lc, "vec": v32[eids], "x": x[nodes], "theta": th,
-             "g": g[nodes], "gg_x": ggx[nodes], "gg_vec": ggv[eids]}
+        a = {"rowptr": lrp, "col": lc, "vec": f64(v32[eids]), "x": f64(x[nodes]), "theta": th,
+             "g": f64(g[nodes]), "gg_x": f64(ggx[nodes]), "gg_vec": f64(ggv[eids])}
         return (kind, args.config, args.family, a), (recvs, nodes, eids)
 
     def edges_of_recv(r):
@@ -417,12 +426,12 @@ def parity_check(args, work, graph, procs, k):
         if kind in ("recv", "recv_dbl", "send", "send_dbl"):
             key = {"recv": "out", "recv_dbl": "d_g", "send": "dx", "send_dbl": "d_x"}[kind]
             ref[key].append(res[key][rows])
-            got[key].append(gpu[key][part])
+            got[key].append(gpu_rows(key, part))
         else:
             order = np.argsort(eids)  # back to the sampled (sorted) edge order
             for key in ("dvec", "d_vec"):
                 ref[key].append(res[key][order])
-                got[key].append(gpu[key][np.sort(eids)])
+                got[key].append(gpu_rows(key, np.sort(eids)))
     errs = {}
     for key in ref:
         rr, gg = np.concatenate(ref[key]), np.concatenate(got[key])

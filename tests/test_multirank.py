@@ -1,6 +1,13 @@
-"""The multi-rank path of the benchmark on CPU: two gloo ranks, each with its
-own graph (weak scaling, no data-path collective), reduced to one whole-job
-figure = edges of all ranks / slowest rank's step time."""
+"""Multi-rank paths on CPU with gloo ranks.
+
+* Replicas: two ranks, each with its own graph (weak scaling, no data-path
+  collective), reduced to one whole-job figure = edges of all ranks / slowest
+  rank's step time.
+* One graph sharded by receiver ranges (2 and 3 ranks): the assembled results
+  of forward, backward and double backward equal the single-rank fp64 oracle.
+* Failure on the host: a rank that leaves between operations makes the peer's
+  next collective end with an error within the process group's timeout.
+"""
 
 import importlib.util
 import os
@@ -180,3 +187,56 @@ def test_receiver_sharded_graph_matches_single_rank(world):
     for k in ref:
         scale = max(np.abs(ref[k]).max(), 1e-30)
         assert np.abs(got[k] - ref[k]).max() / scale < 1e-12, k
+
+
+def _shard_rank_leaves(rank, world, port, q):
+    """Rank 1 leaves before the backward's collectives (between operations,
+    nothing in flight); rank 0's next collective must end with an error within
+    the process group's timeout instead of waiting for good."""
+    import datetime
+    import time
+
+    import torch
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=3))
+    from equivariant_gnn_tensor_receiver_b200.sharded import ShardedConv
+    prob, (rowptr, col, vec), (x, th, g, ggx, ggv, ggt) = _shard_inputs()
+    sc = ShardedConv(rowptr, col, rank, world, None)
+    lg = sc.local
+    sc.ops = _OracleOps(prob, vec[lg.edges])
+    T = lambda a: torch.as_tensor(np.ascontiguousarray(a))
+    lo, hi = lg.lo, lg.hi
+    sc.forward(T(x[lo:hi]), T(th))  # both ranks complete one operation
+    if rank == 1:
+        q.put((rank, "left", 0.0))
+        q.close()
+        q.join_thread()  # flush the message, then vanish
+        os._exit(0)  # no destroy_process_group: the peer simply disappears
+    t0 = time.monotonic()
+    try:
+        sc.backward(T(x[lo:hi]), T(th), T(g[lo:hi]))
+        q.put((rank, "completed", time.monotonic() - t0))
+    except Exception as e:  # gloo reports the lost peer or the timeout
+        q.put((rank, "error:" + type(e).__name__, time.monotonic() - t0))
+    q.close()
+    q.join_thread()
+    os._exit(0)
+
+
+def test_sharded_rank_that_leaves_is_detected_by_the_peer():
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_rank_leaves, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict((r, (s, t)) for r, s, t in (q.get(timeout=120) for _ in procs))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res[1][0] == "left"
+    status, waited = res[0]
+    assert status.startswith("error:"), status
+    assert waited < 60.0
