@@ -307,17 +307,19 @@ def parallel_oracle(cfg, family, procs, n_recv, warmup, steps):
                       f"{steps} timed steps"}
 
 
-def _sub_problem(rowptr, col, edges):
+def _sub_problem(rowptr, col, edges, include=()):
     """The listed edges (CSR positions) as a graph of their own: local receivers
-    (sorted) first, then senders that are not receivers; returns
-    (rowptr, col, receivers' global ids, all local nodes' global ids)."""
+    (sorted) first, then senders that are not receivers and the `include`d
+    nodes that neither (isolated ones keep empty segments); returns
+    (rowptr, col, edge ids in local CSR order, receivers' global ids, all local
+    nodes' global ids)."""
     rowptr = np.asarray(rowptr, dtype=np.int64)
     recv_all = np.repeat(np.arange(len(rowptr) - 1), np.diff(rowptr))
     edges = np.sort(np.asarray(edges, dtype=np.int64))
     r = recv_all[edges]
     s = np.asarray(col, dtype=np.int64)[edges]
     recvs = np.unique(r)
-    extra = np.setdiff1d(np.unique(s), recvs)
+    extra = np.setdiff1d(np.union1d(np.unique(s), np.asarray(include, dtype=np.int64)), recvs)
     nodes = np.concatenate([recvs, extra])
     pos = {int(g): i for i, g in enumerate(nodes)}
     lr = np.fromiter((pos[int(v)] for v in r), dtype=np.int64, count=len(r))
@@ -353,39 +355,34 @@ def _parity_worker(job):
     raise ValueError(kind)
 
 
-def parity_check(args, work, graph, procs, k):
-    """Sampled parity of one full step of the workload against the oracle (see --parity-sample)."""
+def sampled_parity(cfg, family, graph, inputs, out_rows, procs, k, seed=12345):
+    """Element-wise parity of sampled rows against the oracle, on sub-graphs
+    the oracle computes exactly: out and d_g of k (k/4) sampled receivers from
+    their in-edges, dx and d_x of sampled senders from their out-edges, dvec
+    and d_vec of sampled edges from the edge alone (with its receiver).
+    inputs: host arrays x, theta, g, gg_x, gg_vec, vec (fp32 as the device
+    holds them); out_rows(key, idx) -> the device result's rows idx (fp64).
+    Returns the max-norm relative error per output."""
     import multiprocessing as mp
-    import torch
-    rowptr, col, vec = graph
-    N, E = work.N, work.E
-    # host inputs stay fp32 views of the pinned buffers; only the rows a job
-    # needs are widened to fp64, and only sampled rows of the outputs come back
-    # from the device (the capacity workload's full arrays are tens of GB)
-    h = {key: v.numpy() for key, v in work.host.items()}
-    x, g, ggx, ggv, v32 = (h[key] for key in ("x", "g", "gg_x", "gg_vec", "vec"))
-    th = h["theta"].astype(np.float64)
+    rowptr, col, _ = graph
+    rp64 = np.asarray(rowptr, dtype=np.int64)
+    col64 = np.asarray(col, dtype=np.int64)
+    N, E = len(rp64) - 1, len(col64)
+    x, g, ggx, ggv, v32 = (inputs[key] for key in ("x", "g", "gg_x", "gg_vec", "vec"))
+    th = np.asarray(inputs["theta"], dtype=np.float64)
     f64 = lambda a: np.asarray(a, dtype=np.float64)
-
-    def gpu_rows(key, idx):
-        t = work.outs[key]
-        return t.index_select(0, torch.as_tensor(idx, dtype=torch.int64, device=t.device)).double().cpu().numpy()
-
-    gpu = {key: work.outs[key].double().cpu().numpy() for key in ("dtheta", "d_theta")}
-    rng = np.random.default_rng(12345)
-    recv_all = np.repeat(np.arange(N), np.diff(np.asarray(rowptr, dtype=np.int64)))
+    rng = np.random.default_rng(seed)
+    k = min(k, N, E)
     k_dbl = max(1, k // 4)
     rs = np.sort(rng.choice(N, k, replace=False))
     ss = np.sort(rng.choice(N, k, replace=False))
     es = np.sort(rng.choice(E, k, replace=False))
-    col64 = np.asarray(col, dtype=np.int64)
-    rp64 = np.asarray(rowptr, dtype=np.int64)
 
-    def job(kind, edges):
-        lrp, lc, eids, recvs, nodes = _sub_problem(rowptr, col, edges)
+    def job(kind, edges, include=()):
+        lrp, lc, eids, recvs, nodes = _sub_problem(rowptr, col, edges, include)
         a = {"rowptr": lrp, "col": lc, "vec": f64(v32[eids]), "x": f64(x[nodes]), "theta": th,
              "g": f64(g[nodes]), "gg_x": f64(ggx[nodes]), "gg_vec": f64(ggv[eids])}
-        return (kind, args.config, args.family, a), (recvs, nodes, eids)
+        return (kind, cfg, family, a), (recvs, nodes, eids)
 
     def edges_of_recv(r):
         return np.concatenate([np.arange(rp64[i], rp64[i + 1]) for i in r]) if len(r) else np.zeros(0, np.int64)
@@ -395,20 +392,19 @@ def parity_check(args, work, graph, procs, k):
 
     split = lambda arr, n: [a for a in np.array_split(arr, n) if len(a)]
     jobs, meta = [], []
-    for part in split(rs, procs):
-        j, m = job("recv", edges_of_recv(part)); jobs.append(j); meta.append(("recv", part, m))
-    for part in split(rs[:k_dbl], procs):
-        j, m = job("recv_dbl", edges_of_recv(part)); jobs.append(j); meta.append(("recv_dbl", part, m))
-    for part in split(ss, procs):
-        j, m = job("send", edges_of_send(part)); jobs.append(j); meta.append(("send", part, m))
-    for part in split(ss[:k_dbl], procs):
-        j, m = job("send_dbl", edges_of_send(part)); jobs.append(j); meta.append(("send_dbl", part, m))
+    for kind, nodes_k, edges_of in (("recv", rs, edges_of_recv), ("recv_dbl", rs[:k_dbl], edges_of_recv),
+                                    ("send", ss, edges_of_send), ("send_dbl", ss[:k_dbl], edges_of_send)):
+        for part in split(nodes_k, procs):
+            j, m = job(kind, edges_of(part), part)
+            jobs.append(j)
+            meta.append((kind, part, m))
     for part in split(es, procs):
-        j, m = job("edge", part); jobs.append(j); meta.append(("edge", part, m))
+        j, m = job("edge", part)
+        jobs.append(j)
+        meta.append(("edge", part, m))
     env = {key: os.environ.get(key) for key in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
     for key in env:
         os.environ[key] = "1"
-    t0 = time.perf_counter()
     try:
         with mp.get_context("spawn").Pool(procs) as pool:
             results = pool.map(_parity_worker, jobs, chunksize=1)
@@ -421,21 +417,42 @@ def parity_check(args, work, graph, procs, k):
     ref = {key: [] for key in ("out", "d_g", "dx", "d_x", "dvec", "d_vec")}
     got = {key: [] for key in ref}
     for (kind, part, (recvs, nodes, eids)), res in zip(meta, results):
-        pos = {int(v): i for i, v in enumerate(nodes)}
-        rows = np.array([pos[int(v)] for v in part])
         if kind in ("recv", "recv_dbl", "send", "send_dbl"):
+            pos = {int(v): i for i, v in enumerate(nodes)}
+            rows = np.array([pos[int(v)] for v in part])
             key = {"recv": "out", "recv_dbl": "d_g", "send": "dx", "send_dbl": "d_x"}[kind]
             ref[key].append(res[key][rows])
-            got[key].append(gpu_rows(key, part))
+            got[key].append(out_rows(key, part))
         else:
             order = np.argsort(eids)  # back to the sampled (sorted) edge order
             for key in ("dvec", "d_vec"):
                 ref[key].append(res[key][order])
-                got[key].append(gpu_rows(key, np.sort(eids)))
+                got[key].append(out_rows(key, np.sort(eids)))
     errs = {}
     for key in ref:
         rr, gg = np.concatenate(ref[key]), np.concatenate(got[key])
         errs[key] = float(np.abs(gg - rr).max() / max(np.abs(rr).max(), 1e-30))
+    return errs, dict(receivers=k, senders=k, edges=k, dbl_nodes=k_dbl)
+
+
+def parity_check(args, work, graph, procs, k):
+    """Sampled parity of one full step of the workload against the oracle (see
+    --parity-sample), plus dTheta / d_Theta by additivity over receiver halves."""
+    import torch
+    N = work.N
+    rp64 = np.asarray(graph[0], dtype=np.int64)
+    # host inputs stay fp32 views of the pinned buffers; only sampled rows of
+    # the outputs come back from the device (the capacity workload's full
+    # arrays are tens of GB)
+    h = {key: v.numpy() for key, v in work.host.items()}
+
+    def gpu_rows(key, idx):
+        t = work.outs[key]
+        return t.index_select(0, torch.as_tensor(idx, dtype=torch.int64, device=t.device)).double().cpu().numpy()
+
+    t0 = time.perf_counter()
+    errs, sampled = sampled_parity(args.config, args.family, graph, h, gpu_rows, procs, k)
+    gpu = {key: work.outs[key].double().cpu().numpy() for key in ("dtheta", "d_theta")}
     # dTheta and d_Theta: the full graph against the sum over its two receiver
     # halves (the library on both sides; additivity holds at any size)
     T = work.T
@@ -459,8 +476,9 @@ def parity_check(args, work, graph, procs, k):
     for key in ("dtheta", "d_theta"):
         errs[key + "_additivity"] = float(np.abs(sums[key] - gpu[key]).max() / max(np.abs(gpu[key]).max(), 1e-30))
     tol = 1e-5 if args.gemm in ("fp32", "simt") else 5e-3
-    return {"parity": args.config, "gemm": args.gemm, "family": args.family, "nodes": N, "edges": E,
-            "sampled_receivers": k, "sampled_senders": k, "sampled_edges": k, "sampled_dbl_nodes": k_dbl,
+    return {"parity": args.config, "gemm": args.gemm, "family": args.family, "nodes": N, "edges": work.E,
+            "sampled_receivers": sampled["receivers"], "sampled_senders": sampled["senders"],
+            "sampled_edges": sampled["edges"], "sampled_dbl_nodes": sampled["dbl_nodes"],
             "max_norm_rel_err": errs, "tolerance": tol, "pass": all(v < tol for v in errs.values()),
             "oracle_s": round(time.perf_counter() - t0, 1), "oracle_procs": procs}
 

@@ -31,59 +31,113 @@
 
 namespace tpc {
 
-// Q[m1][m3] += a[m1] c[m3] on the structural nonzeros of the coupling matrix
-template <int L1, int L2, int L3>
-__device__ __forceinline__ void outer_Q(const float* a, const float* c, float* Q) {
+// ---- one path restricted to the output components m3 in [A3, B3) -------------
+// The per-lane state of a path (coupling rows M, Md and the accumulators Q, Qh)
+// has one entry per structural nonzero (m1, m3).  Large paths (l = 3 with
+// 26-42 nonzeros) run their channel loop in two passes over halves of the m3
+// range, each holding only its half of that state: the same arithmetic, half
+// the registers.  TriPart compresses the nonzeros of the restricted range.
+template <int L1, int L2, int L3, int A3, int B3>
+struct TriPart {
+  using TR = Tri<L1, L2, L3>;
+  static constexpr int N1 = TR::N1, N2 = TR::N2, N3 = TR::N3;
+  struct Tab {
+    bool m[N1][N3];
+    int mi[N1][N3];
+    int nmz;
+  };
+  static constexpr Tab make() {
+    Tab t{};
+    int c = 0;
+    for (int a = 0; a < N1; ++a)
+      for (int b = 0; b < N3; ++b) {
+        const bool on = TR::tab.m[a][b] && b >= A3 && b < B3;
+        t.m[a][b] = on;
+        t.mi[a][b] = on ? c++ : -1;
+      }
+    t.nmz = c;
+    return t;
+  }
+  static constexpr Tab tab = make();
+  static constexpr int NMZ = tab.nmz > 0 ? tab.nmz : 1;
+};
+
+// Mrow[mi] = sum_m2 C[m1,m2,m3] Y[m2] on the part's nonzeros
+template <class TP, int L1, int L2, int L3>
+__device__ __forceinline__ void part_coupling_row(const float* Y, float* Mrow) {
   using TR = Tri<L1, L2, L3>;
   sfor<TR::N1>([&](auto I1) {
     sfor<TR::N3>([&](auto I3) {
       constexpr int i1 = decltype(I1)::value, i3 = decltype(I3)::value;
-      if constexpr (TR::tab.m[i1][i3]) {
-        constexpr int mi = TR::tab.mi[i1][i3];
+      if constexpr (TP::tab.m[i1][i3]) {
+        float s = 0.f;
+        sfor<TR::N2>([&](auto I2) {
+          constexpr int i2 = decltype(I2)::value;
+          if constexpr (TR::tab.cg[i1][i2][i3]) s = fmaf(TR::template cg<i1, i2, i3>(), Y[i2], s);
+        });
+        constexpr int mi = TP::tab.mi[i1][i3];
+        Mrow[mi] = s;
+      }
+    });
+  });
+}
+// T[m3] = sum_m1 M[m1][m3] x[m1] for the part's m3 (other entries zero)
+template <class TP>
+__device__ __forceinline__ void part_apply_M(const float* Mv, const float* xv, float* T) {
+#pragma unroll
+  for (int i3 = 0; i3 < TP::N3; ++i3) T[i3] = 0.f;
+  sfor<TP::N1>([&](auto I1) {
+    sfor<TP::N3>([&](auto I3) {
+      constexpr int i1 = decltype(I1)::value, i3 = decltype(I3)::value;
+      if constexpr (TP::tab.m[i1][i3]) {
+        constexpr int mi = TP::tab.mi[i1][i3];
+        T[i3] = fmaf(Mv[mi], xv[i1], T[i3]);
+      }
+    });
+  });
+}
+// (T, Td)[m3] = sum_m1 (M, Md)[m1][m3] x[m1], and T1[m3] = sum_m1 M[m1][m3] x1[m1]
+template <class TP>
+__device__ __forceinline__ void part_apply_M2(const float2* MM, const float* xv, const float* x1v, float2* TT,
+                                              float* T1) {
+#pragma unroll
+  for (int i3 = 0; i3 < TP::N3; ++i3) {
+    TT[i3] = make_float2(0.f, 0.f);
+    T1[i3] = 0.f;
+  }
+  sfor<TP::N1>([&](auto I1) {
+    sfor<TP::N3>([&](auto I3) {
+      constexpr int i1 = decltype(I1)::value, i3 = decltype(I3)::value;
+      if constexpr (TP::tab.m[i1][i3]) {
+        constexpr int mi = TP::tab.mi[i1][i3];
+        TT[i3] = __ffma2_rn(MM[mi], make_float2(xv[i1], xv[i1]), TT[i3]);
+        T1[i3] = fmaf(MM[mi].x, x1v[i1], T1[i3]);
+      }
+    });
+  });
+}
+// Q[mi] += a[m1] c[m3] on the part's nonzeros
+template <class TP>
+__device__ __forceinline__ void part_outer_Q(const float* a, const float* c, float* Q) {
+  sfor<TP::N1>([&](auto I1) {
+    sfor<TP::N3>([&](auto I3) {
+      constexpr int i1 = decltype(I1)::value, i3 = decltype(I3)::value;
+      if constexpr (TP::tab.m[i1][i3]) {
+        constexpr int mi = TP::tab.mi[i1][i3];
         Q[mi] = fmaf(a[i1], c[i3], Q[mi]);
       }
     });
   });
 }
-
-// (Q[mi], Q'[mi]) += (a[m1], a'[m1]) c[m3] on the structural nonzeros
-template <int L1, int L2, int L3>
-__device__ __forceinline__ void outer_Q2(const float* a, const float* a2, const float* c, float2* QQ) {
+// out[m2] += sum_{m1, m3 in the part} C[m1,m2,m3] Q[m1][m3]
+template <class TP, int L1, int L2, int L3>
+__device__ __forceinline__ void part_contract_Q(const float* Q, float* out) {
   using TR = Tri<L1, L2, L3>;
   sfor<TR::N1>([&](auto I1) {
     sfor<TR::N3>([&](auto I3) {
       constexpr int i1 = decltype(I1)::value, i3 = decltype(I3)::value;
-      if constexpr (TR::tab.m[i1][i3]) {
-        constexpr int mi = TR::tab.mi[i1][i3];
-        QQ[mi] = __ffma2_rn(make_float2(a[i1], a2[i1]), make_float2(c[i3], c[i3]), QQ[mi]);
-      }
-    });
-  });
-}
-// Q[mi] += a[m1] c[m3] into the first members of QQ
-template <int L1, int L2, int L3>
-__device__ __forceinline__ void outer_Q_first(const float* a, const float* c, float2* QQ) {
-  using TR = Tri<L1, L2, L3>;
-  sfor<TR::N1>([&](auto I1) {
-    sfor<TR::N3>([&](auto I3) {
-      constexpr int i1 = decltype(I1)::value, i3 = decltype(I3)::value;
-      if constexpr (TR::tab.m[i1][i3]) {
-        constexpr int mi = TR::tab.mi[i1][i3];
-        QQ[mi].x = fmaf(a[i1], c[i3], QQ[mi].x);
-      }
-    });
-  });
-}
-
-// out[m2] += sum_{m1,m3} C[m1,m2,m3] Q[m1][m3]
-template <int L1, int L2, int L3>
-__device__ __forceinline__ void contract_Q(const float* Q, float* out) {
-  using TR = Tri<L1, L2, L3>;
-  sfor<TR::N1>([&](auto I1) {
-    sfor<TR::N3>([&](auto I3) {
-      constexpr int i1 = decltype(I1)::value, i3 = decltype(I3)::value;
-      if constexpr (TR::tab.m[i1][i3]) {
-        constexpr int mi = TR::tab.mi[i1][i3];
+      if constexpr (TP::tab.m[i1][i3]) {
+        constexpr int mi = TP::tab.mi[i1][i3];
         sfor<TR::N2>([&](auto I2) {
           constexpr int i2 = decltype(I2)::value;
           if constexpr (TR::tab.cg[i1][i2][i3]) out[i2] = fmaf(TR::template cg<i1, i2, i3>(), Q[mi], out[i2]);
@@ -92,6 +146,47 @@ __device__ __forceinline__ void contract_Q(const float* Q, float* out) {
     });
   });
 }
+// float pairs J0 .. J0+NP-1 of a 16-byte aligned shared array: 16-byte reads
+// where the pair index is even, 8-byte reads otherwise (J0, NP compile-time)
+template <int J0, int NP>
+__device__ __forceinline__ void lds_f2_at(const float* base, float2* v) {
+  if constexpr (NP > 0) {
+    if constexpr ((J0 & 1) == 0 && NP >= 2) {
+      const float4 t = lds4(base + 2 * J0);
+      v[0] = make_float2(t.x, t.y);
+      v[1] = make_float2(t.z, t.w);
+      lds_f2_at<J0 + 2, NP - 2>(base, v + 2);
+    } else {
+      v[0] = *reinterpret_cast<const float2*>(base + 2 * J0);
+      lds_f2_at<J0 + 1, NP - 1>(base, v + 1);
+    }
+  }
+}
+// floats OFF .. OFF+N-1 of a 16-byte aligned shared array, in the widest reads
+// their alignment allows (OFF, N compile-time)
+template <int OFF, int N>
+__device__ __forceinline__ void lds_run(const float* base, float* v) {
+  if constexpr (N > 0) {
+    if constexpr ((OFF & 3) == 0 && N >= 4) {
+      const float4 t = lds4(base + OFF);
+      v[0] = t.x;
+      v[1] = t.y;
+      v[2] = t.z;
+      v[3] = t.w;
+      lds_run<OFF + 4, N - 4>(base, v + 4);
+    } else if constexpr ((OFF & 1) == 0 && N >= 2) {
+      const float2 t = *reinterpret_cast<const float2*>(base + OFF);
+      v[0] = t.x;
+      v[1] = t.y;
+      lds_run<OFF + 2, N - 2>(base, v + 2);
+    } else {
+      v[0] = base[OFF];
+      lds_run<OFF + 1, N - 1>(base, v + 1);
+    }
+  }
+}
+// the m3 halves of a path: split when its per-lane state exceeds this many nonzeros
+constexpr int kWnaSplitNmz = 24;
 
 // Shared G tiles hold radial pairs side by side, [u][k / 2][m3][k & 1], so that a
 // 16-byte read yields float2 operands (G_2kp, G_2kp+1) for paired FMAs.
@@ -100,21 +195,24 @@ __host__ __device__ constexpr int g_slot(int k, int m3) {
   return ((k >> 1) * N3 + m3) * 2 + (k & 1);
 }
 
-// one path of one 32-edge batch (GT: the second order has a Gt operand)
-// rfirst: chunk-local receiver of lane 0's edge; the window's receivers are
-// rfirst .. rfirst + nslots - 1 and the lane's is rfirst + myslot (myslot < 0:
-// no edge).
-template <int L1, int L2, int L3, int RM, bool DBL, bool GT>
+// one path of one 32-edge batch, output components m3 in [A3, B3) (GT: the
+// second order has a Gt operand).  rfirst: chunk-local receiver of lane 0's
+// edge; the window's receivers are rfirst .. rfirst + nslots - 1 and the lane's
+// is rfirst + myslot (myslot < 0: no edge).  db, hb collect over all parts.
+template <int L1, int L2, int L3, int RM, bool DBL, bool GT, bool XB, int A3, int B3>
 __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, const WnaLay& L, float* ws, int rfirst,
                                          int nslots, int myslot, int nc, int nb, int myrow,
                                          const float* __restrict__ x,
                                          const float* __restrict__ x1, const float* __restrict__ G,
                                          const float* __restrict__ Gt, float2* db, float2* hb) {
   using TR = Tri<L1, L2, L3>;
-  constexpr int N1 = TR::N1, N2 = TR::N2, N3 = TR::N3, NMZ = TR::NMZ, GW = RM * N3, NK2 = RM / 2;
+  using TP = TriPart<L1, L2, L3, A3, B3>;
+  constexpr int N1 = TR::N1, N2 = TR::N2, N3 = TR::N3, NMZ = TP::NMZ, GW = RM * N3, NK2 = RM / 2;
+  constexpr int NH = B3 - A3;  // m3 components of this part
   constexpr int CH = kWnChunk;
   static_assert(CH == 4, "the chunk is one group of four channels");
-  constexpr int NIT = (GW * CH + 31) / 32;  // G elements per lane and chunk (upper bound)
+  static_assert(0 <= A3 && A3 < B3 && B3 <= N3, "m3 part");
+  constexpr int NIT = (RM * NH * CH + 31) / 32;  // G elements of the part per lane and chunk (upper bound)
   const int lane = lane_id();
   const float* geo = ws + L.Geo + lane * L.geos;
   // first order: M in Mv; second order: (M, Md) side by side in MM (paired FMAs);
@@ -126,14 +224,14 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
     float Y[N2], Mrow[NMZ];
 #pragma unroll
     for (int i = 0; i < N2; ++i) Y[i] = geo[L2 * L2 + i];
-    coupling_row<L1, L2, L3>(Y, DBL ? Mrow : Mv);
+    part_coupling_row<TP, L1, L2, L3>(Y, DBL ? Mrow : Mv);
 #pragma unroll
     for (int kp = 0; kp < NK2; ++kp) b2[kp] = make_float2(geo[16 + 2 * kp], geo[17 + 2 * kp]);
     if constexpr (DBL) {
       float Mdrow[NMZ];
 #pragma unroll
       for (int i = 0; i < N2; ++i) Y[i] = geo[16 + RM + L2 * L2 + i];
-      coupling_row<L1, L2, L3>(Y, Mdrow);
+      part_coupling_row<TP, L1, L2, L3>(Y, Mdrow);
 #pragma unroll
       for (int i = 0; i < NMZ; ++i) MM[i] = make_float2(Mrow[i], Mdrow[i]);
 #pragma unroll
@@ -153,8 +251,9 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
   const int Kb = pl.Kb[q.i3];
   constexpr bool has_t = DBL && GT;
   const bool has_x1 = DBL && x1 != nullptr;
-  // this lane's G elements of a chunk: source offset (relative to receiver row
-  // and channel u0) and position inside a slot, the same for every chunk
+  // this lane's G elements of a chunk (the part's m3 only): source offset
+  // (relative to receiver row and channel u0) and position inside a slot, the
+  // same for every chunk
   constexpr int NS = kWnaSlots(DBL);
   const size_t rowstride = size_t(N3) * Kb;
   const float* Gp = G + size_t(nc) * pl.a_pref[q.i3] + size_t(rfirst) * rowstride + q.koff;
@@ -163,8 +262,8 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
 #pragma unroll
   for (int it = 0; it < NIT; ++it) {
     const int t = it * 32 + lane;
-    const int u = t & (CH - 1), km = t / CH;  // km = k * N3 + m3
-    const int k = km / N3, m3 = km - k * N3;
+    const int u = t & (CH - 1), km = t / CH;  // km = k * NH + (m3 - A3)
+    const int k = km / NH, m3 = A3 + (km - k * NH);
     gsrc[it] = k < R ? m3 * Kb + k * c + u : -1;
     gdst[it] = u * GW + g_slot<N3>(k, m3);
   }
@@ -215,39 +314,64 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
     __syncwarp();
     const float* sG = active ? ws + L.G + (ch & 1) * L.gbuf + (myslot - g0) * L.gslot : ws + L.Z;
     const float* sGt = active ? ws + L.Gt + (ch & 1) * L.gbuf + (myslot - g0) * L.gslot : ws + L.Z;
-    // the lane's four channels in N1 16-byte reads
-    float xg[CH * N1], x1g[DBL ? CH * N1 : 1];
-    lds_vec<CH * N1>(ws + L.X + (ch & 1) * L.xbuf + lane * L.xs, xg);
-    if constexpr (DBL) lds_vec<CH * N1>(ws + L.X1 + (ch & 1) * L.xbuf + lane * L.xs, x1g);
+    // the lane's rows of the four channels: all at once in N1 16-byte reads, or
+    // in kernels with l = 3 features channel by channel (one channel's x, x1
+    // live at a time)
+    constexpr bool XBULK = XB;
+    const float* sXl = ws + L.X + (ch & 1) * L.xbuf + lane * L.xs;
+    const float* sX1l = ws + L.X1 + (ch & 1) * L.xbuf + lane * L.xs;
+    float xg[XBULK ? CH * N1 : 1], x1g[XBULK && DBL ? CH * N1 : 1];
+    if constexpr (XBULK) {
+      lds_vec<CH * N1>(sXl, xg);
+      if constexpr (DBL) lds_vec<CH * N1>(sX1l, x1g);
+    }
+    sfor<CH>([&](auto TI) {
+      constexpr int t = decltype(TI)::value;
+      float xv[N1];
+      if constexpr (XBULK) {
 #pragma unroll
-    for (int t = 0; t < CH; ++t) {
-      const float* xv = xg + t * N1;
+        for (int i = 0; i < N1; ++i) xv[i] = xg[t * N1 + i];
+      } else {
+        lds_run<t * N1, N1>(sXl, xv);
+      }
       if constexpr (!DBL) {
         float T[N3];
-        apply_M<L1, L2, L3>(Mv, xv, T);
-        float2 g2[NK2 * N3];
-        lds_f2<NK2 * N3>(sG + t * GW, g2);
+        part_apply_M<TP>(Mv, xv, T);
+        float2 g2[NK2 * NH];
+        if constexpr (NH == N3) {
+          lds_f2_at<0, NK2 * N3>(sG + t * GW, g2);
+        } else {
+          sfor<NK2>([&](auto KP) {
+            constexpr int kp = decltype(KP)::value;
+            lds_f2_at<kp * N3 + A3, NH>(sG + t * GW, g2 + kp * NH);
+          });
+        }
         float2 dT2[N3];
 #pragma unroll
-        for (int i = 0; i < N3; ++i) dT2[i] = make_float2(0.f, 0.f);
+        for (int i = A3; i < B3; ++i) dT2[i] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int kp = 0; kp < NK2; ++kp)
 #pragma unroll
-          for (int i = 0; i < N3; ++i) {
-            const float2 g = g2[kp * N3 + i];
+          for (int i = A3; i < B3; ++i) {
+            const float2 g = g2[kp * NH + (i - A3)];
             dT2[i] = __ffma2_rn(b2[kp], g, dT2[i]);
             db[kp] = __ffma2_rn(g, make_float2(T[i], T[i]), db[kp]);
           }
         float dT[N3];
 #pragma unroll
-        for (int i = 0; i < N3; ++i) dT[i] = dT2[i].x + dT2[i].y;
-        outer_Q<L1, L2, L3>(xv, dT, Q);
+        for (int i = 0; i < N3; ++i) dT[i] = (i >= A3 && i < B3) ? dT2[i].x + dT2[i].y : 0.f;
+        part_outer_Q<TP>(xv, dT, Q);
       } else {
-        const float* x1v = x1g + t * N1;
+        float x1v[N1];
+        if constexpr (XBULK) {
+#pragma unroll
+          for (int i = 0; i < N1; ++i) x1v[i] = x1g[t * N1 + i];
+        } else {
+          lds_run<t * N1, N1>(sX1l, x1v);
+        }
         float2 TT[N3];  // (M x, Md x)
-        apply_M2<L1, L2, L3>(MM, xv, TT);
         float T[N3], T12[N3];
-        apply_M_first<L1, L2, L3>(MM, x1v, T12);
+        part_apply_M2<TP>(MM, xv, x1v, TT, T12);
 #pragma unroll
         for (int i = 0; i < N3; ++i) {
           T[i] = TT[i].x;
@@ -255,60 +379,92 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
         }
         float2 dG2[N3], dX2[N3];
 #pragma unroll
-        for (int i = 0; i < N3; ++i) dG2[i] = dX2[i] = make_float2(0.f, 0.f);
+        for (int i = A3; i < B3; ++i) dG2[i] = dX2[i] = make_float2(0.f, 0.f);
         // G (and Gt) rows in KH slices of radial pairs (bounds the live registers)
         constexpr int KH = NK2 >= 4 ? 2 : 1, KS = NK2 / KH;  // KS pairs per slice
-#pragma unroll
-        for (int kh = 0; kh < KH; ++kh) {
-          float2 g2[KS * N3], gt2[GT ? KS * N3 : 1];
-          lds_f2<KS * N3>(sG + t * GW + 2 * kh * KS * N3, g2);
-          if constexpr (GT) lds_f2<KS * N3>(sGt + t * GW + 2 * kh * KS * N3, gt2);
+        sfor<KH>([&](auto KHI) {
+          constexpr int kh = decltype(KHI)::value;
+          float2 g2[KS * NH];
+          [[maybe_unused]] float2 gt2[GT ? KS * NH : 1];
+          if constexpr (NH == N3) {
+            lds_f2_at<kh * KS * N3, KS * N3>(sG + t * GW, g2);
+            if constexpr (GT) lds_f2_at<kh * KS * N3, KS * N3>(sGt + t * GW, gt2);
+          } else {
+            sfor<KS>([&](auto KK) {
+              constexpr int kk = decltype(KK)::value, kp = kh * KS + kk;
+              lds_f2_at<kp * N3 + A3, NH>(sG + t * GW, g2 + kk * NH);
+              if constexpr (GT) lds_f2_at<kp * N3 + A3, NH>(sGt + t * GW, gt2 + kk * NH);
+            });
+          }
 #pragma unroll
           for (int kk = 0; kk < KS; ++kk) {
             const int kp = kh * KS + kk;
 #pragma unroll
-            for (int i = 0; i < N3; ++i) {
-              const float2 g = g2[kk * N3 + i];
+            for (int i = A3; i < B3; ++i) {
+              const float2 g = g2[kk * NH + (i - A3)];
               dG2[i] = __ffma2_rn(b2[kp], g, dG2[i]);
               dX2[i] = __ffma2_rn(bd2[kp], g, dX2[i]);
               db[kp] = __ffma2_rn(g, make_float2(T12[i], T12[i]), db[kp]);
               hb[kp] = __ffma2_rn(g, make_float2(T[i], T[i]), hb[kp]);
               if constexpr (GT) {
-                const float2 gt = gt2[kk * N3 + i];
+                const float2 gt = gt2[kk * NH + (i - A3)];
                 dX2[i] = __ffma2_rn(b2[kp], gt, dX2[i]);
                 db[kp] = __ffma2_rn(gt, make_float2(T[i], T[i]), db[kp]);
               }
             }
           }
-        }
+        });
         float dG[N3], dX[N3];
 #pragma unroll
         for (int i = 0; i < N3; ++i) {
-          dG[i] = dG2[i].x + dG2[i].y;
-          dX[i] = dX2[i].x + dX2[i].y;
+          dG[i] = (i >= A3 && i < B3) ? dG2[i].x + dG2[i].y : 0.f;
+          dX[i] = (i >= A3 && i < B3) ? dX2[i].x + dX2[i].y : 0.f;
         }
-        outer_Q<L1, L2, L3>(x1v, dG, Q);
-        outer_Q<L1, L2, L3>(xv, dX, Q);
-        outer_Q<L1, L2, L3>(xv, dG, Qh);
+        part_outer_Q<TP>(x1v, dG, Q);
+        part_outer_Q<TP>(xv, dX, Q);
+        part_outer_Q<TP>(xv, dG, Qh);
       }
-    }
+    });
     __syncwarp();
   }
   }  // receiver groups
-  // this path's share of dY (second order: wY, hY) for the lane's edge
+  // this part's share of dY (second order: wY, hY) for the lane's edge
   float* acc = ws + L.Acc + lane * L.accs;
   float o[N2];
 #pragma unroll
   for (int i = 0; i < N2; ++i) o[i] = 0.f;
-  contract_Q<L1, L2, L3>(Q, o);
+  part_contract_Q<TP, L1, L2, L3>(Q, o);
 #pragma unroll
   for (int i = 0; i < N2; ++i) acc[L2 * L2 + i] += o[i];
   if constexpr (DBL) {
 #pragma unroll
     for (int i = 0; i < N2; ++i) o[i] = 0.f;
-    contract_Q<L1, L2, L3>(Qh, o);
+    part_contract_Q<TP, L1, L2, L3>(Qh, o);
 #pragma unroll
     for (int i = 0; i < N2; ++i) acc[16 + L2 * L2 + i] += o[i];
+  }
+}
+
+// one path of one batch: whole, or in two m3 parts when its per-lane state is
+// large.  The instantiation with the gg_Theta operand (GT) keeps whole paths: its
+// split form gave wrong d_vec on the warps of a CTA other than the first, for
+// plans that mix l = 0 and l = 3 blocks, and no cause was found in the code.
+template <int L1, int L2, int L3, int RM, bool DBL, bool GT, bool XB>
+__device__ __forceinline__ void wna_path_parts(const DevPlan& pl, const DevPath& q, const WnaLay& L, float* ws,
+                                               int rfirst, int nslots, int myslot, int nc, int nb, int myrow,
+                                               const float* __restrict__ x, const float* __restrict__ x1,
+                                               const float* __restrict__ G, const float* __restrict__ Gt, float2* db,
+                                               float2* hb) {
+  constexpr int N3 = 2 * L3 + 1;
+  if constexpr (Tri<L1, L2, L3>::NMZ > kWnaSplitNmz && N3 >= 3 && !(DBL && GT)) {
+    constexpr int H = (N3 + 1) / 2;
+    wna_path<L1, L2, L3, RM, DBL, GT, XB, 0, H>(pl, q, L, ws, rfirst, nslots, myslot, nc, nb, myrow, x, x1, G, Gt, db,
+                                            hb);
+    wna_path<L1, L2, L3, RM, DBL, GT, XB, H, N3>(pl, q, L, ws, rfirst, nslots, myslot, nc, nb, myrow, x, x1, G, Gt, db,
+                                             hb);
+  } else {
+    wna_path<L1, L2, L3, RM, DBL, GT, XB, 0, N3>(pl, q, L, ws, rfirst, nslots, myslot, nc, nb, myrow, x, x1, G, Gt, db,
+                                             hb);
   }
 }
 
@@ -434,8 +590,8 @@ __global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
 #define TPC_CASE(a, b, c)                                                                                 \
   case triple_id(a, b, c):                                                                                \
     if constexpr (a <= LF && c <= LF)                                                                     \
-      wna_path<a, b, c, RM, DBL, GT>(pl, q, L, ws, rfirst, nslots, myslot, nc, nb, myrow, x, x1, G, Gt, db2, \
-                                     hb2);                                                                \
+      wna_path_parts<a, b, c, RM, DBL, GT, (LF <= 2)>(pl, q, L, ws, rfirst, nslots, myslot, nc, nb, myrow, x, x1, G, Gt, \
+                                           db2, hb2);                                                     \
     break;
           TPC_FOR_EACH_TRIPLE(TPC_CASE)
 #undef TPC_CASE
