@@ -384,10 +384,11 @@ int tpconv_plan_create(tpconv_plan** out, const char* irreps_in, int l_sh_max,
     d.wn_smem_s = wn_smem_bytes(d.rm, d.wn_cpl, d.n3max, d.nmz_max, false, false);
     d.wn_smem_f2 = wn_smem_bytes(d.rm, 1, d.n1max, d.nmz_max, true, true);
     d.wn_smem_s2 = wn_smem_bytes(d.rm, 1, d.n3max, d.nmz_max, true, false);
-    d.wn_smem_adj = wna_smem_bytes(d.rm, d.n3max, d.n1max, false);
-    d.wn_smem_dadj = wna_smem_bytes(d.rm, d.n3max, d.n1max, true);
+    d.wn_smem_adj = wna_smem_bytes(d.rm, d.n3max, d.n1max, false, false);
+    d.wn_smem_dadj = wna_smem_bytes(d.rm, d.n3max, d.n1max, true, false);
+    const int dadj_gt = wna_smem_bytes(d.rm, d.n3max, d.n1max, true, true);  // launcher computes it again
     const int mx = std::max(std::max(std::max(d.wn_smem_f, d.wn_smem_s), std::max(d.wn_smem_f2, d.wn_smem_s2)),
-                            std::max(d.wn_smem_adj, d.wn_smem_dadj));
+                            std::max(std::max(d.wn_smem_adj, d.wn_smem_dadj), dadj_gt));
     if (mx > 227 * 1024) {
       delete p;
       return TPCONV_ERR_UNSUPPORTED;

@@ -185,8 +185,10 @@ __device__ __forceinline__ void lds_run(const float* base, float* v) {
     }
   }
 }
-// the m3 halves of a path: split when its per-lane state exceeds this many nonzeros
-constexpr int kWnaSplitNmz = 24;
+// the m3 halves of a path: split when its per-lane state exceeds this many
+// nonzeros (second order with l = 3 features: a lower bound, as their x rows
+// and coupling rows are longer)
+constexpr int kWnaSplitNmz = 24, kWnaSplitNmzL3 = 16;
 
 // Shared G tiles hold radial pairs side by side, [u][k / 2][m3][k & 1], so that a
 // 16-byte read yields float2 operands (G_2kp, G_2kp+1) for paired FMAs.
@@ -254,7 +256,7 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
   // this lane's G elements of a chunk (the part's m3 only): source offset
   // (relative to receiver row and channel u0) and position inside a slot, the
   // same for every chunk
-  constexpr int NS = kWnaSlots(DBL);
+  const int NS = L.ns;
   const size_t rowstride = size_t(N3) * Kb;
   const float* Gp = G + size_t(nc) * pl.a_pref[q.i3] + size_t(rfirst) * rowstride + q.koff;
   const float* Gtp = has_t ? Gt + (Gp - G) : nullptr;
@@ -301,8 +303,8 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
   };
 
   // receivers in groups of NS slots (one group unless the window spans more
-  // than NS receivers); a lane whose receiver is not in the group reads the
-  // zero slot, which adds nothing to its sums
+  // than NS receivers); a lane whose receiver is not in the group adds nothing
+  // (its x rows read as zero)
   for (g0 = 0; g0 < nslots; g0 += NS) {
   const bool active = myslot >= g0 && myslot < g0 + NS;
   if (nch > 0) stage(0);
@@ -312,14 +314,18 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
     ac_commit();
     ac_wait<1>();
     __syncwarp();
-    const float* sG = active ? ws + L.G + (ch & 1) * L.gbuf + (myslot - g0) * L.gslot : ws + L.Z;
-    const float* sGt = active ? ws + L.Gt + (ch & 1) * L.gbuf + (myslot - g0) * L.gslot : ws + L.Z;
+    // a lane whose receiver is not in this group reads slot 0 and the zero x row
+    const int sl = active ? myslot - g0 : 0;  // lanes without an edge (myslot < 0) read slot 0 too
+    const float* sG = ws + L.G + (ch & 1) * L.gbuf + sl * L.gslot;
+    const float* sGt = ws + L.Gt + (ch & 1) * L.gbuf + sl * L.gslot;
     // the lane's rows of the four channels: all at once in N1 16-byte reads, or
     // in kernels with l = 3 features channel by channel (one channel's x, x1
     // live at a time)
     constexpr bool XBULK = XB;
-    const float* sXl = ws + L.X + (ch & 1) * L.xbuf + lane * L.xs;
-    const float* sX1l = ws + L.X1 + (ch & 1) * L.xbuf + lane * L.xs;
+    // (first order: one group, every lane with an edge is in it)
+    const bool xz = DBL && !active;
+    const float* sXl = xz ? ws + L.XZ : ws + L.X + (ch & 1) * L.xbuf + lane * L.xs;
+    const float* sX1l = xz ? ws + L.XZ : ws + L.X1 + (ch & 1) * L.xbuf + lane * L.xs;
     float xg[XBULK ? CH * N1 : 1], x1g[XBULK && DBL ? CH * N1 : 1];
     if constexpr (XBULK) {
       lds_vec<CH * N1>(sXl, xg);
@@ -456,7 +462,8 @@ __device__ __forceinline__ void wna_path_parts(const DevPlan& pl, const DevPath&
                                                const float* __restrict__ G, const float* __restrict__ Gt, float2* db,
                                                float2* hb) {
   constexpr int N3 = 2 * L3 + 1;
-  if constexpr (Tri<L1, L2, L3>::NMZ > kWnaSplitNmz && N3 >= 3 && !(DBL && GT)) {
+  constexpr int split_nmz = XB || !DBL ? kWnaSplitNmz : kWnaSplitNmzL3;  // XB: kernels with l <= 2
+  if constexpr (Tri<L1, L2, L3>::NMZ > split_nmz && N3 >= 3 && !(DBL && GT)) {
     constexpr int H = (N3 + 1) / 2;
     wna_path<L1, L2, L3, RM, DBL, GT, XB, 0, H>(pl, q, L, ws, rfirst, nslots, myslot, nc, nb, myrow, x, x1, G, Gt, db,
                                             hb);
@@ -489,10 +496,10 @@ __global__ void __launch_bounds__(32 * kWnWarps, DBL ? 2 : 3)
              float* __restrict__ dbout, const int* __restrict__ extra, int* __restrict__ counter) {
   extern __shared__ __align__(16) float sm[];
   const int warp = threadIdx.x >> 5, lane = lane_id();
-  const WnaLay L = wna_layout_of(RM, pl.n3max, pl.n1max, DBL);
+  const WnaLay L = wna_layout_of(RM, pl.n3max, pl.n1max, DBL, GT);
   float* ws = sm + warp * L.total;
   int& s_base = *reinterpret_cast<int*>(sm + kWnWarps * L.total);  // this round's first item
-  // staged buffers read where nothing was staged (and the zero slot) must hold zeros
+  // staged buffers read where nothing was staged (radial entries k >= R) must hold zeros
   for (int i = lane; i < L.Geo; i += 32) ws[i] = 0.f;
   const int e_lo = rowptr[r0], e_hi = rowptr[r0 + nc];
   const int total = DBL ? (e_hi - e_lo + kBatchEdges - 1) / kBatchEdges : nc + extra[nc];

@@ -48,50 +48,60 @@ TPC_HD inline int wn_smem_bytes(int RM, int cpl, int nimax, int nmz_max, bool db
 
 // ---- lane = edge (receiver adjoint streams, first and second order) --------
 // Second order: a warp's lanes are 32 consecutive CSR edges, which may belong
-// to several receivers; the G rows of up to kWnaSlots(true) of them are staged
-// at once.  First order: a warp's lanes are up to 32 edges of one receiver
-// (one slot).
-// G, Gt : two chunk buffers, each kWnaSlots slots of kWnChunk channels of one
-//         receiver's G (and Gt), [u][k/2][m3][k&1] with row stride
-//         RM * (2 l3 + 1) of the path (zero where never staged); slot stride
-//         gslot = kWnChunk * gs + 4 floats, so that lanes reading different
-//         slots fall into different bank quads
-// Z     : one slot of zeros, read by lanes whose receiver is not staged
+// to several receivers; the G rows of up to `ns` of them are staged at once (a
+// window spanning more receivers runs its channel loop once per group of ns).
+// First order: a warp's lanes are up to 32 edges of one receiver (one slot).
+// G, Gt : two chunk buffers, each ns slots of kWnChunk channels of one
+//         receiver's G (and Gt, only with the gg_Theta operand),
+//         [u][k/2][m3][k&1] with row stride RM * (2 l3 + 1) of the path (zero
+//         where never staged); slot stride gslot = kWnChunk * gs + 4 floats, so
+//         that lanes reading different slots fall into different bank quads
 // X, X1 : two chunk buffers of the 32 lanes' rows, [lane][u * n1 + m1] with row
 //         stride xs, xs / 4 odd: the 16-byte reads of 8 consecutive lanes fall
 //         into distinct bank quads
 // Geo   : per lane Y[16], b[RM] (and Yd[16], bd[RM]), odd stride
 // Acc   : per lane accumulators that persist across paths (dY, or wY and hY), odd stride
-TPC_HD constexpr int kWnaSlots(bool dbl) { return dbl ? 2 : 1; }
+// XZ    : one row of zeros (xs floats); a lane whose receiver is not in the group
+//         being staged reads it for its x rows (and any staged G slot), which
+//         makes every term it adds zero.
+//
+// ns: 1 for the first order; for the second order 2 with the Gt operand, else
+// 3 when the slices of three slots still let two CTAs share an SM (the same
+// rule on host and device), else 2.
+constexpr int kWnaTwoCtaBytes = (228 * 1024 - 2 * 1024) / 2;  // dynamic shared memory of one of two CTAs per SM
 struct WnaLay {
-  int G, Gt, Z, X, X1, Geo, Acc;
-  int gs, gslot, gbuf, xs, xbuf, geos, accs;
+  int G, Gt, X, X1, XZ, Geo, Acc;
+  int ns, gs, gslot, gbuf, xs, xbuf, geos, accs;
   int total;
 };
 
-TPC_HD inline WnaLay wna_layout_of(int RM, int n3max, int n1max, bool dbl) {
+TPC_HD inline WnaLay wna_layout_of(int RM, int n3max, int n1max, bool dbl, bool gt) {
   WnaLay L;
   L.gs = RM * n3max;
   L.gslot = kWnChunk * L.gs + 4;
-  L.gbuf = kWnaSlots(dbl) * L.gslot;
   L.xs = (kWnChunk * n1max + 3) & ~3;
   if ((L.xs >> 2) % 2 == 0) L.xs += 4;
   L.xbuf = 32 * L.xs;
   L.geos = (dbl ? 2 : 1) * (16 + RM) + 1;
   L.accs = (dbl ? 32 : 16) + 1;
-  L.G = 0;
-  L.Gt = L.G + 2 * L.gbuf;
-  L.Z = L.Gt + (dbl ? 2 * L.gbuf : 0);
-  L.X = L.Z + L.gslot;
-  L.X1 = L.X + 2 * L.xbuf;
-  L.Geo = L.X1 + (dbl ? 2 * L.xbuf : 0);
-  L.Acc = L.Geo + 32 * L.geos;
-  L.total = (L.Acc + 32 * L.accs + 3) & ~3;
+  for (int ns = dbl ? (gt ? 2 : 3) : 1;; --ns) {
+    L.ns = ns;
+    L.gbuf = ns * L.gslot;
+    L.G = 0;
+    L.Gt = L.G + 2 * L.gbuf;
+    L.X = L.Gt + (gt ? 2 * L.gbuf : 0);
+    L.X1 = L.X + 2 * L.xbuf;
+    L.XZ = L.X1 + (dbl ? 2 * L.xbuf : 0);
+    L.Geo = L.XZ + L.xs;
+    L.Acc = L.Geo + 32 * L.geos;
+    L.total = (L.Acc + 32 * L.accs + 3) & ~3;
+    if (ns <= 2 || kWnWarps * L.total * 4 + 16 <= kWnaTwoCtaBytes) break;
+  }
   return L;
 }
 // the warps' slices and one int (the CTA's batch count)
-TPC_HD inline int wna_smem_bytes(int RM, int n3max, int n1max, bool dbl) {
-  return kWnWarps * wna_layout_of(RM, n3max, n1max, dbl).total * 4 + 16;
+TPC_HD inline int wna_smem_bytes(int RM, int n3max, int n1max, bool dbl, bool gt) {
+  return kWnWarps * wna_layout_of(RM, n3max, n1max, dbl, gt).total * 4 + 16;
 }
 
 // ---- work items of the streams (lists built in graph.cuh) ----
