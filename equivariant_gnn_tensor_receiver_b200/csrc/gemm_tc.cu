@@ -78,8 +78,8 @@ struct TcAcc {
 template <int BN, bool SPLIT>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const __grid_constant__ CUtensorMap tmBlo, int M, int N, int K, TcOut out, int accumulate,
-              uint64_t limit) {
+              const __grid_constant__ CUtensorMap tmBlo, const __grid_constant__ CUtensorMap tmC, int M, int N,
+              int K, TcOut out, int accumulate, int tma_out, uint64_t limit) {
   using SM = TcSmem<BN>;
   constexpr int S = SM::kStages;
   constexpr uint32_t kCols = TcAcc<BN, SPLIT>::kCols;
@@ -232,7 +232,36 @@ __global__ void __launch_bounds__(192, 1)
       const int nrounds = (nk + RS::D - 1) / RS::D;
       while (ok && drained < nrounds) ok = drain(drained);
     }
-    if (ok) {
+    // plain row-major output (tma_out): the tile goes through the operand ring,
+    // idle once every MMA has completed, as BN / 32 boxes of 128 rows x 128 bytes
+    // in the 128-byte swizzle, and leaves by TMA stores
+    if (tma_out && !ok) *abort_flag = 1;
+    if (ok && tma_out) {
+      const int r = q * 32 + lane;
+      const int nacc = nk < NACC ? nk : NACC;
+#pragma unroll
+      for (int c = 0; c < BN; c += 16) {
+        float v[16];
+        if constexpr (DRAIN) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = racc[(c + i) % NR];
+        } else {
+          tmem_ld16(tlane + uint32_t(c), v);
+          for (int a = 1; a < nacc; ++a) {
+            float w[16];
+            tmem_ld16(tlane + uint32_t(a * kCols + c), w);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] += w[i];
+          }
+        }
+        float* box = reinterpret_cast<float*>(base + (c / 32) * (kBM * 128));
+        const int j0 = (c % 32) / 4;  // first 16-byte chunk of these 16 columns in the box row
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          *reinterpret_cast<float4*>(box + r * 32 + (((j0 + i) ^ (r & 7)) * 4)) =
+              make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      }
+    } else if (ok) {
       const int row = m0 + q * 32 + lane;
       const int64_t rbase = (row / out.rdiv) * out.r_hi + (row % out.rdiv) * out.r_lo;
       const int nacc = nk < NACC ? nk : NACC;  // accumulators that received a K step
@@ -279,6 +308,17 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       }
+    }
+  }
+  if (tma_out && warp >= 2) {
+    // every epilogue thread's writes are visible to the async proxy before one
+    // thread stores the boxes; all four warps pass the barrier whatever happened
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (threadIdx.x == 64 && !*abort_flag) {
+#pragma unroll 1
+      for (int b = 0; b < BN / 32; ++b) tma_store_2d(&tmC, base + b * (kBM * 128), n0 + 32 * b, m0);
+      tma_store_commit_and_wait_read();  // the boxes stay in shared memory until read
     }
   }
   // drain: the producer waits (bounded) for the loads it issued so no copy is
@@ -332,13 +372,18 @@ bool make_map(CUtensorMap* m, const float* p, int64_t rows, int64_t cols, int64_
 template <int BN, bool SPLIT>
 cudaError_t run(const float* A, int64_t lda, const float* B, const float* Blo, int64_t ldb, int M, int N, int K,
                 TcOut out, int accumulate, uint64_t limit, cudaStream_t st) {
-  CUtensorMap ta, tb, tbl;
+  CUtensorMap ta, tb, tbl, tc;
   if (!make_map(&ta, A, M, K, lda, kBM) || !make_map(&tb, B, N, K, ldb, BN)) return cudaErrorInvalidValue;
   if (SPLIT && !make_map(&tbl, Blo, N, K, ldb, BN)) return cudaErrorInvalidValue;
   if (!SPLIT) tbl = tb;
+  // a plain row-major output C[i][j] = p[i * r_hi + j], written (not added), leaves by TMA stores
+  const int tma_out = !accumulate && out.rdiv == 1 && out.r_lo == 0 && out.c_hi == 1 &&
+                      make_map(&tc, out.p, M, N, out.r_hi, kBM);
+  if (!tma_out) tc = ta;
   using SM = TcSmem<BN>;
+  static_assert(BN / 32 * kBM * 128 <= SM::kStages * SM::kStage, "the output tile fits the operand ring");
   dim3 grid(unsigned((M + kBM - 1) / kBM), unsigned((N + BN - 1) / BN));
-  k_gemm_tc<BN, SPLIT><<<grid, 192, SM::kBytes, st>>>(ta, tb, tbl, M, N, K, out, accumulate, limit);
+  k_gemm_tc<BN, SPLIT><<<grid, 192, SM::kBytes, st>>>(ta, tb, tbl, tc, M, N, K, out, accumulate, tma_out, limit);
   return cudaGetLastError();
 }
 
