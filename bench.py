@@ -627,7 +627,7 @@ def roofline(T, plan, prof_ms, E):
         ach = flops / (prof_ms[dom] * 1e-3) / 1e12
         peak = N_SM * FP32_LANES_PER_SM * 2 * sm_max * 1e6 / 1e12
         roof.update(bound="alu", achieved=ach, peak=peak, unit="TFLOP/s", frac=ach / peak,
-                    peak_source=f"148 SM x 128 FP32 lanes x 2 x {sm_max:.0f} MHz (max clock, {peak_src} file)",
+                    peak_source=f"148 SM x 128 FP32 lanes x 2 x {sm_max:.0f} MHz (max SM clock, {peak_src} peaks)",
                     work=f"{wm[dom]} algorithmic FMA per edge x {E} edges")
     try:
         with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
