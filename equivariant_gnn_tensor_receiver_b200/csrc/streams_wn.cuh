@@ -297,8 +297,16 @@ __device__ __forceinline__ void wn_chan_path(const DevPlan& pl, const DevPath& q
 // them (second launch, which starts after the first has finished).
 // RECV: ptr = rowptr, nbr = col (edge id = CSR position); else ptr = s_rowptr,
 // nbr = s_recv, perm = sender-sorted position -> edge id.
+// CTAs per SM the register budget is sized for: the second-order forms with
+// l = 3 features hold 2 by shared memory (their coupling rows and staged rows
+// are longer), so they get the registers of 2
+template <int LF, bool RECV, bool DBL>
+constexpr int wn_min_ctas() {
+  return DBL && LF >= 3 ? 2 : (DBL && RECV ? 3 : 4);
+}
+
 template <int RM, int LF, int CPL, bool RECV, bool DBL, bool P1, bool EXTRA>
-__global__ void __launch_bounds__(32 * kWnWarps, DBL && RECV ? 3 : 4)
+__global__ void __launch_bounds__(32 * kWnWarps, wn_min_ctas<LF, RECV, DBL>())
     k_wn_stream(const __grid_constant__ DevPlan pl, int n0, int nc, const int* __restrict__ ptr,
                 const int* __restrict__ nbr, const int* __restrict__ perm, const float* __restrict__ vec,
                 const float* __restrict__ ggv, const float* __restrict__ src, const float* __restrict__ src1,
