@@ -54,12 +54,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, uint64_t
   return false;
 }
 
+// Column tiles of at most 64 run two CTAs per SM (two stages each: the same
+// bytes in flight per SM as one CTA with four, in two independent pipelines,
+// and twice the CTA slots for the partial waves); wider tiles one CTA.
+template <int BN>
+constexpr int tc_ctas_per_sm() {
+  return BN <= 64 ? 2 : 1;
+}
+
 template <int BN>
 struct TcSmem {
   static constexpr int kA = kBM * kBK * 4;   // 16 KB
   static constexpr int kB = BN * kBK * 4;    // BN x 128 B
   static constexpr int kStage = 2 * kA + 2 * kB;
-  static constexpr int kStages = (200 * 1024) / kStage >= 4 ? 4 : ((200 * 1024) / kStage >= 3 ? 3 : 2);
+  static constexpr int kStages = tc_ctas_per_sm<BN>() == 2
+                                     ? 2
+                                     : ((200 * 1024) / kStage >= 4 ? 4 : ((200 * 1024) / kStage >= 3 ? 3 : 2));
   static constexpr int kBytes = kStages * kStage + 1024 /*align*/ + 256 /*barriers: 3 x stages + 5, slot, flag*/;
 };
 
@@ -70,13 +80,15 @@ struct TcSmem {
 template <int BN, bool SPLIT>
 struct TcAcc {
   static constexpr int kCols = BN < 32 ? 32 : BN;
-  static constexpr int N = SPLIT ? (512 / kCols > 8 ? 8 : 512 / kCols) : 1;
+  // TMEM columns of one CTA: 512 / (CTAs per SM)
+  static constexpr int kMaxCols = 512 / tc_ctas_per_sm<BN>();
+  static constexpr int N = SPLIT ? (kMaxCols / kCols > 8 ? 8 : kMaxCols / kCols) : 1;
   static constexpr uint32_t kAlloc = kCols * N;  // power of two, <= 512
   static constexpr bool kDrain = SPLIT && BN <= 128;
 };
 
 template <int BN, bool SPLIT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, tc_ctas_per_sm<BN>())
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmBlo, const __grid_constant__ CUtensorMap tmC, int M, int N,
               int K, TcOut out, int accumulate, int tma_out, uint64_t limit) {
