@@ -58,7 +58,7 @@ using namespace tc;
 constexpr int kBM = 128, kBK = 32;
 constexpr int kMaxMaps = 2 * kMaxBlocks;   // (pair, input block)
 constexpr int kMaxGroups = 2 * kMaxPaths;  // (pair, path)
-constexpr int kMaxSms = 160;               // partial buffer: two waves on up to this many SMs
+constexpr int kMaxSms = 160;               // partial buffer: two tiles per SM on up to this many SMs
 
 int64_t sm_count() {
   int dev = 0, n = 148;
@@ -87,12 +87,18 @@ struct __align__(64) DtParams {
   uint64_t wait_ns;
 };
 
+// Column tiles of at most 64 run two CTAs per SM (two stages and four TMEM
+// accumulators each), wider tiles one; the planner sizes the split for that.
+constexpr int dt_ctas_per_sm(int bn) { return bn <= 64 ? 2 : 1; }
+
 template <int BN>
 struct DtSmem {
   static constexpr int kA = kBM * kBK * 4;  // 16 KB: four 32 x 32 boxes
   static constexpr int kB = BN * kBK * 4;
   static constexpr int kStage = 2 * kA + 2 * kB;
-  static constexpr int kStages = (200 * 1024) / kStage >= 4 ? 4 : ((200 * 1024) / kStage >= 3 ? 3 : 2);
+  static constexpr int kStages = dt_ctas_per_sm(BN) == 2
+                                     ? 2
+                                     : ((200 * 1024) / kStage >= 4 ? 4 : ((200 * 1024) / kStage >= 3 ? 3 : 2));
   static constexpr int kBytes = kStages * kStage + 1024 + 256;
 };
 
@@ -102,7 +108,8 @@ struct DtSmem {
 template <int BN, bool SPLIT>
 struct DtAcc {
   static constexpr int kCols = BN < 32 ? 32 : BN;
-  static constexpr int N = SPLIT ? (512 / kCols > 8 ? 8 : 512 / kCols) : 1;
+  static constexpr int kMaxCols = 512 / dt_ctas_per_sm(BN);  // TMEM columns of one CTA
+  static constexpr int N = SPLIT ? (kMaxCols / kCols > 8 ? 8 : kMaxCols / kCols) : 1;
   static constexpr uint32_t kAlloc = kCols * N;
   static constexpr bool kDrain = SPLIT && BN <= 128;
 };
@@ -115,7 +122,7 @@ __device__ __forceinline__ bool waitp(uint64_t* b, uint32_t parity, uint64_t lim
 }
 
 template <int BN, bool SPLIT>
-__global__ void __launch_bounds__(192, 1) k_dtheta_tc(const __grid_constant__ DtParams P) {
+__global__ void __launch_bounds__(192, dt_ctas_per_sm(BN)) k_dtheta_tc(const __grid_constant__ DtParams P) {
   using SM = DtSmem<BN>;
   constexpr int S = SM::kStages;
   constexpr uint32_t kCols = DtAcc<BN, SPLIT>::kCols;
@@ -542,7 +549,7 @@ cudaError_t dtheta_tc_accumulate(const DevPlan& d, int s0, int nc, const float* 
   for (int i = 0; i < ng; ++i) Kmax = std::max<int64_t>(Kmax, gr[i].K);
   Kmax = (Kmax + 31) & ~int64_t(31);
   const int64_t cap = int64_t(dtheta_tc_partial_floats(d) / (size_t(BN) * kBM));
-  const int64_t sms = sm_count();
+  const int64_t sms = sm_count() * dt_ctas_per_sm(BN);  // CTA slots of one wave
   int64_t best_kc = -1, best_cost = 0;
   for (int64_t kc = 32; kc <= Kmax; kc += 32) {
     const int64_t n = count(kc);
