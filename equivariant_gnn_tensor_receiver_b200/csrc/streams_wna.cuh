@@ -214,6 +214,13 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
   constexpr int CH = kWnChunk;
   static_assert(CH == 4, "the chunk is one group of four channels");
   static_assert(0 <= A3 && A3 < B3 && B3 <= N3, "m3 part");
+  // channels of a chunk unrolled together: the second-order bodies unroll two
+  // (a runtime loop over the pairs), which halves their code against four
+  // unrolled channels; instruction fetch stalls were 0.7 cycles per issue with
+  // four.  Measured second-order adjoint: mace-like layer 2.29 -> 2.22 ms,
+  // sweep at degree 25 2.90 -> 2.71 ms, wide layer 27.1 -> 26.4 ms (one
+  // channel at a time: 2.38, 2.64, 28.2 ms).
+  constexpr int CHU = DBL ? 2 : CH;
   constexpr int NIT = (RM * NH * CH + 31) / 32;  // G elements of the part per lane and chunk (upper bound)
   const int lane = lane_id();
   const float* geo = ws + L.Geo + lane * L.geos;
@@ -326,19 +333,25 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
     const bool xz = DBL && !active;
     const float* sXl = xz ? ws + L.XZ : ws + L.X + (ch & 1) * L.xbuf + lane * L.xs;
     const float* sX1l = xz ? ws + L.XZ : ws + L.X1 + (ch & 1) * L.xbuf + lane * L.xs;
-    float xg[XBULK ? CH * N1 : 1], x1g[XBULK && DBL ? CH * N1 : 1];
-    if constexpr (XBULK) {
+    constexpr bool XB4 = XBULK && CHU == CH;  // bulk x loads need the four channels unrolled
+    float xg[XB4 ? CH * N1 : 1], x1g[XB4 && DBL ? CH * N1 : 1];
+    if constexpr (XB4) {
       lds_vec<CH * N1>(sXl, xg);
       if constexpr (DBL) lds_vec<CH * N1>(sX1l, x1g);
     }
-    sfor<CH>([&](auto TI) {
-      constexpr int t = decltype(TI)::value;
+    // one channel t of the chunk (compile-time when the whole chunk is unrolled)
+    auto chan = [&](auto TI, int tg) {
+      constexpr int ti = decltype(TI)::value;
+      const int t = CHU == CH ? ti : tg + ti;
       float xv[N1];
-      if constexpr (XBULK) {
+      if constexpr (CHU < CH) {
 #pragma unroll
-        for (int i = 0; i < N1; ++i) xv[i] = xg[t * N1 + i];
+        for (int i = 0; i < N1; ++i) xv[i] = sXl[t * N1 + i];
+      } else if constexpr (XB4) {
+#pragma unroll
+        for (int i = 0; i < N1; ++i) xv[i] = xg[ti * N1 + i];
       } else {
-        lds_run<t * N1, N1>(sXl, xv);
+        lds_run<ti * N1, N1>(sXl, xv);
       }
       if constexpr (!DBL) {
         float T[N3];
@@ -369,11 +382,14 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
         part_outer_Q<TP>(xv, dT, Q);
       } else {
         float x1v[N1];
-        if constexpr (XBULK) {
+        if constexpr (CHU < CH) {
 #pragma unroll
-          for (int i = 0; i < N1; ++i) x1v[i] = x1g[t * N1 + i];
+          for (int i = 0; i < N1; ++i) x1v[i] = sX1l[t * N1 + i];
+        } else if constexpr (XB4) {
+#pragma unroll
+          for (int i = 0; i < N1; ++i) x1v[i] = x1g[ti * N1 + i];
         } else {
-          lds_run<t * N1, N1>(sX1l, x1v);
+          lds_run<ti * N1, N1>(sX1l, x1v);
         }
         float2 TT[N3];  // (M x, Md x)
         float T[N3], T12[N3];
@@ -430,7 +446,13 @@ __device__ __forceinline__ void wna_path(const DevPlan& pl, const DevPath& q, co
         part_outer_Q<TP>(xv, dX, Q);
         part_outer_Q<TP>(xv, dG, Qh);
       }
-    });
+    };
+    if constexpr (CHU == CH) {
+      sfor<CH>([&](auto TI) { chan(TI, 0); });
+    } else {
+#pragma unroll 1
+      for (int tg = 0; tg < CH; tg += CHU) sfor<CHU>([&](auto TI) { chan(TI, tg); });
+    }
     __syncwarp();
   }
   }  // receiver groups
