@@ -666,8 +666,10 @@ def per_direction(work, steps, flush):
             "dbl_edges_per_s": E / (t_d * 1e-3), "fwd_ms": t_f, "fwd_bwd_ms": t_fb, "dbl_ms": t_d}
 
 
-def roofline(T, plan, prof_ms, E):
-    """FP32-ALU roofline of the dominant phase (algorithmic FMAs, see work_model)."""
+def roofline(T, plan, prof_ms, E, workload_key):
+    """FP32-ALU roofline of the dominant phase (algorithmic FMAs, see work_model).
+    `traffic` comes from the ncu record of that phase only when the record was
+    taken on this workload (config, family, gemm) and on the current sources."""
     peaks, peak_src = measured_peaks()
     wm = work_model(T, plan)
     dom = max(prof_ms, key=lambda k: prof_ms[k])
@@ -684,7 +686,7 @@ def roofline(T, plan, prof_ms, E):
     try:
         with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
             tr = json.load(f).get(dom)
-        if tr and tr.get("sources_sha256") == sources_digest(tr["sources"]):
+        if tr and tr.get("workload") == workload_key and tr.get("sources_sha256") == sources_digest(tr["sources"]):
             roof["traffic"] = tr["dram_bytes_per_launch"]
             roof["traffic_kernel"] = tr["kernel"]
     except (OSError, ValueError):
@@ -742,7 +744,8 @@ def run_suite(args):
                 **{k: v for k, v in pd.items()},
                 "step_edges_per_s": w.E / (t_step * 1e-3), "step_ms": t_step,
                 "peak_mem_bytes": peak, "workspace_bytes": w.ws_bytes, "inputs_bytes": inputs,
-                "outputs_bytes": outputs, "roofline": roofline(T, w.plan, prof_ms, w.E),
+                "outputs_bytes": outputs,
+                "roofline": roofline(T, w.plan, prof_ms, w.E, f"{cfg}/{args.family}/{gemm}"),
                 "phases_ms": {k: round(v, 4) for k, v in prof_ms.items() if v > 0}}
         print(json.dumps(line), flush=True)
         del w
@@ -880,7 +883,7 @@ def run_ours(args):
 
     # roofline of the dominant phase
     phase_ms = {k: ms / args.steps for k, (ms, _) in prof.items()}
-    roof = roofline(T, plan, phase_ms, E)
+    roof = roofline(T, plan, phase_ms, E, f"{args.config}/{args.family}/{args.gemm}")
 
     per_dir = per_direction(work, args.steps, flush)
     for k in ("fwd_ms", "fwd_bwd_ms", "dbl_ms"):  # slowest rank; every rank takes the same steps

@@ -100,3 +100,26 @@ def test_sampled_parity_end_to_end_with_isolated_nodes():
     assert sampled["receivers"] == N  # every node sampled, isolated ones included
     assert set(errs) == {"out", "d_g", "dx", "d_x", "dvec", "d_vec"}
     assert max(errs.values()) < 1e-12, errs
+
+
+def test_traffic_record_applies_only_to_its_workload():
+    """The ncu DRAM-traffic figure of the dominant phase is reported only for the
+    workload (config / family / gemm) and the sources it was captured on."""
+    import json
+    B = _bench()
+    import equivariant_gnn_tensor_receiver_b200 as T
+    c = W.CONFIGS["mace"]
+    plan = T.Plan(c["irreps_in"], c["l_sh_max"], c["irreps_out"], c["R"], radial=c["radial"],
+                  radial_params=c["radial_params"])
+    with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+        rec = json.load(f)["dbl_edge_r"]
+    prof = {"fwd_edge": 0.6, "dbl_edge_r": 2.2, "bwd_edge_r": 1.3}
+    own = B.roofline(T, plan, prof, 213738, rec["workload"])
+    other = B.roofline(T, plan, prof, 213738, "wide/full/fp32")
+    assert own["phase"] == other["phase"] == "dbl_edge_r"
+    if rec["sources_sha256"] == B.sources_digest(rec["sources"]):
+        assert own["traffic"] == rec["dram_bytes_per_launch"] and own["traffic_kernel"] == rec["kernel"]
+    else:  # the kernel changed since the capture: no traffic figure at all
+        assert own["traffic"] is None
+    assert other["traffic"] is None and "traffic_kernel" not in other
+    assert own["frac"] == other["frac"] and 0 < own["frac"] < 1
